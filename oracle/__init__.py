@@ -1,0 +1,148 @@
+"""fp64 CPU oracle for the Parallax decode forward.
+
+TEST INFRASTRUCTURE ONLY: imported by tests/, by the smoke check and by the
+bench's CPU-baseline leg. The product path (the CUDA library and its binding)
+never imports it and shares no code with it.
+
+Every function takes arrays in the product layout and widens them to float64
+(exact for bf16 and fp32 inputs):
+    q, r, out : [B, Hq, D]
+    k, v      : [B, Hkv, Lmax, D]
+    seqlens   : [B] int32, each in [0, Lmax]
+
+The arithmetic lives in parallax_oracle.c; its header gives the equations and
+the passages of the pages they follow.
+"""
+import ctypes
+
+import numpy as np
+
+from . import build as _build
+
+
+def _f64(x):
+    if hasattr(x, "detach"):  # torch tensor: widen on the host, exactly
+        x = x.detach().cpu().double().numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _ptr(a, ctype=ctypes.c_double):
+    return a.ctypes.data_as(ctypes.POINTER(ctype))
+
+
+class Oracle:
+    """The oracle functions of one compiled copy of parallax_oracle.c."""
+
+    def __init__(self, path):
+        lib = ctypes.CDLL(path)
+        dp = ctypes.POINTER(ctypes.c_double)
+        ip = ctypes.POINTER(ctypes.c_int32)
+        i = ctypes.c_int
+        d = ctypes.c_double
+        lib.oracle_parallax_covariance.argtypes = [dp, dp, dp, dp, ip, i, i, i, i, i, d, dp]
+        lib.oracle_parallax_expanded.argtypes = [dp, dp, dp, dp, ip, i, i, i, i, i, d, dp]
+        lib.oracle_parallax_streaming.argtypes = [dp, dp, dp, dp, ip, i, i, i, i, i, d, i, dp]
+        lib.oracle_softmax_decode.argtypes = [dp, dp, dp, ip, i, i, i, i, i, d, dp]
+        for f in (lib.oracle_parallax_covariance, lib.oracle_parallax_expanded,
+                  lib.oracle_parallax_streaming, lib.oracle_softmax_decode,
+                  lib.oracle_num_threads):
+            f.restype = ctypes.c_int
+        self._lib = lib
+        self.path = path
+
+    @staticmethod
+    def _prep(q, k, v, seqlens):
+        q, k, v = _f64(q), _f64(k), _f64(v)
+        if hasattr(seqlens, "detach"):
+            seqlens = seqlens.detach().cpu().numpy()
+        seqlens = np.ascontiguousarray(np.asarray(seqlens, dtype=np.int32))
+        if q.ndim != 3 or k.ndim != 4 or v.shape != k.shape:
+            raise ValueError("expected q [B,Hq,D] and k, v [B,Hkv,Lmax,D]")
+        B, Hq, D = q.shape
+        _, Hkv, Lmax, Dk = k.shape
+        if k.shape[0] != B or Dk != D or seqlens.shape != (B,):
+            raise ValueError("shape mismatch between q, k, v and seqlens")
+        return q, k, v, seqlens, B, Hq, Hkv, Lmax, D
+
+    @staticmethod
+    def _check(rc, name):
+        if rc != 0:
+            raise ValueError(f"{name} rejected its arguments (rc={rc})")
+
+    def _parallax(self, fn, name, q, r, k, v, seqlens, scale, *extra):
+        q, k, v, seqlens, B, Hq, Hkv, Lmax, D = self._prep(q, k, v, seqlens)
+        r = _f64(r)
+        if r.shape != q.shape:
+            raise ValueError("r must have the shape of q")
+        out = np.zeros((B, Hq, D))
+        rc = fn(_ptr(q), _ptr(r), _ptr(k), _ptr(v), _ptr(seqlens, ctypes.c_int32),
+                B, Hq, Hkv, Lmax, D, float(scale), *extra, _ptr(out))
+        self._check(rc, name)
+        return out
+
+    def parallax_covariance(self, q, r, k, v, seqlens, scale):
+        """o = vbar + sum_i w_i (s_i - sbar)(v_i - vbar): the definition form."""
+        return self._parallax(self._lib.oracle_parallax_covariance,
+                              "oracle_parallax_covariance", q, r, k, v, seqlens, scale)
+
+    def parallax_expanded(self, q, r, k, v, seqlens, scale):
+        """o = A/l + C/l - (b/l)(A/l) with l, A, b, C summed over all keys."""
+        return self._parallax(self._lib.oracle_parallax_expanded,
+                              "oracle_parallax_expanded", q, r, k, v, seqlens, scale)
+
+    def parallax_streaming(self, q, r, k, v, seqlens, scale, chunk):
+        """Online accumulators over chunks of `chunk` keys, merged by max-rescaling."""
+        return self._parallax(self._lib.oracle_parallax_streaming,
+                              "oracle_parallax_streaming", q, r, k, v, seqlens, scale,
+                              int(chunk))
+
+    def softmax_decode(self, q, k, v, seqlens, scale):
+        """Plain softmax attention, the R = 0 special case."""
+        q, k, v, seqlens, B, Hq, Hkv, Lmax, D = self._prep(q, k, v, seqlens)
+        out = np.zeros((B, Hq, D))
+        rc = self._lib.oracle_softmax_decode(_ptr(q), _ptr(k), _ptr(v),
+                                             _ptr(seqlens, ctypes.c_int32), B, Hq, Hkv,
+                                             Lmax, D, float(scale), _ptr(out))
+        self._check(rc, "oracle_softmax_decode")
+        return out
+
+    # The default used by parity checks: the definition (covariance) form.
+    def parallax_decode(self, q, r, k, v, seqlens, scale):
+        return self.parallax_covariance(q, r, k, v, seqlens, scale)
+
+    def num_threads(self) -> int:
+        return int(self._lib.oracle_num_threads())
+
+
+_default = None
+
+
+def default() -> Oracle:
+    global _default
+    if _default is None:
+        _default = Oracle(_build.build())
+    return _default
+
+
+def parallax_covariance(*a, **kw):
+    return default().parallax_covariance(*a, **kw)
+
+
+def parallax_expanded(*a, **kw):
+    return default().parallax_expanded(*a, **kw)
+
+
+def parallax_streaming(*a, **kw):
+    return default().parallax_streaming(*a, **kw)
+
+
+def softmax_decode(*a, **kw):
+    return default().softmax_decode(*a, **kw)
+
+
+def parallax_decode(*a, **kw):
+    return default().parallax_decode(*a, **kw)
+
+
+def num_threads() -> int:
+    return default().num_threads()

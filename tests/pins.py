@@ -1,0 +1,278 @@
+"""Pins for the fp64 oracle: facts fixed by the pages or by mathematics.
+
+Each pin takes an `oracle.Oracle` and raises AssertionError when the oracle
+disagrees with something that does not come from the oracle itself:
+  - hand-worked examples (tests/golden/hand_examples.txt);
+  - the R = 0 identity with softmax attention, checked against torch's own
+    softmax and matmul ("Integrazioni AI personalizzate dopo l'attenzione
+    Parallax", encorp.ai, FAQ: zero projection gives softmax attention);
+  - the local-linear reading: with the probe set to the LLA solver output
+    Sigma_w^{-1}(q - kbar), the output equals the intercept of the weighted
+    least-squares line, solved here by numpy's lstsq ("Parallax: Parameterized
+    Local Linear Attention for Language Modeling", bayesiansapien blog,
+    opening diagram: LLA is the local linear estimate);
+  - closed forms, invariances and brute-force agreement between the forms.
+
+test_oracle_pins.py runs them on the real oracle; test_oracle_mutants.py
+checks that each planted mistake in a copy of the oracle trips one of them.
+"""
+import math
+import os
+
+import numpy as np
+import torch
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+FORMS = ("covariance", "expanded", "streaming3", "streaming1")
+
+
+def run_form(orc, form, q, r, k, v, n, scale):
+    if form == "covariance":
+        return orc.parallax_covariance(q, r, k, v, n, scale)
+    if form == "expanded":
+        return orc.parallax_expanded(q, r, k, v, n, scale)
+    if form == "streaming3":
+        return orc.parallax_streaming(q, r, k, v, n, scale, 3)
+    if form == "streaming1":
+        return orc.parallax_streaming(q, r, k, v, n, scale, 1)
+    raise ValueError(form)
+
+
+def all_forms(orc, q, r, k, v, n, scale):
+    return {f: run_form(orc, f, q, r, k, v, n, scale) for f in FORMS}
+
+
+def rand_case(seed, B=2, Hq=4, Hkv=2, D=8, Lmax=24, lengths=(11, 24), r_scale=0.5):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((B, Hq, D))
+    r = rng.standard_normal((B, Hq, D)) * r_scale
+    k = rng.standard_normal((B, Hkv, Lmax, D))
+    v = rng.standard_normal((B, Hkv, Lmax, D))
+    n = np.array(lengths, dtype=np.int32)
+    return q, r, k, v, n
+
+
+def close(a, b, tol=1e-11, what=""):
+    a, b = np.asarray(a), np.asarray(b)
+    err = np.max(np.abs(a - b) / np.maximum(1.0, np.abs(b))) if a.size else 0.0
+    assert np.all(np.isfinite(a)), f"{what}: non-finite output"
+    assert err <= tol, f"{what}: max scaled error {err:.3e} > {tol:.1e}"
+
+
+# ---------------------------------------------------------------- golden ----
+
+def load_hand_examples():
+    examples, cur = [], None
+    with open(os.path.join(GOLDEN, "hand_examples.txt")) as f:
+        for line in f:
+            line = line.split("#", 1)[0].strip()
+            if not line:
+                continue
+            key, val = (x.strip() for x in line.split("=", 1))
+            if key == "name":
+                cur = {"name": val, "k": [], "v": []}
+                examples.append(cur)
+            elif key in ("k", "v"):
+                cur[key].append([float(x) for x in val.split()])
+            elif key == "scale":
+                cur[key] = float(val)
+            else:
+                cur[key] = [float(x) for x in val.split()]
+    return examples
+
+
+def pin_hand_examples(orc):
+    for ex in load_hand_examples():
+        n = len(ex["k"])
+        q = np.array(ex["q"])[None, None, :]
+        r = np.array(ex["r"])[None, None, :]
+        k = np.array(ex["k"])[None, None, :, :]
+        v = np.array(ex["v"])[None, None, :, :]
+        want = np.array(ex["o"])[None, None, :]
+        for form, got in all_forms(orc, q, r, k, v, [n], ex["scale"]).items():
+            close(got, want, 1e-12, f"{ex['name']} ({form})")
+        if not np.any(r):
+            close(orc.softmax_decode(q, k, v, [n], ex["scale"]), want, 1e-12,
+                  f"{ex['name']} (softmax)")
+
+
+# ------------------------------------------------------ R = 0 is softmax ----
+
+def torch_softmax_attention(q, k, v, n, scale):
+    """softmax(scale q K^T) V per head with torch's own routines (fp64)."""
+    q, k, v = (torch.from_numpy(np.asarray(x, dtype=np.float64)) for x in (q, k, v))
+    B, Hq, D = q.shape
+    G = Hq // k.shape[1]
+    kk = torch.repeat_interleave(k, G, dim=1)  # [B, Hq, Lmax, D]
+    vv = torch.repeat_interleave(v, G, dim=1)
+    out = torch.zeros(B, Hq, D, dtype=torch.float64)
+    for b in range(B):
+        nb = int(n[b])
+        if nb == 0:
+            continue
+        logits = scale * torch.einsum("hd,hld->hl", q[b], kk[b, :, :nb])
+        out[b] = torch.einsum("hl,hld->hd", torch.softmax(logits, dim=-1), vv[b, :, :nb])
+    return out.numpy()
+
+
+def pin_r_zero_is_softmax(orc):
+    q, r, k, v, n = rand_case(1, B=3, Hq=6, Hkv=2, D=16, Lmax=40, lengths=(17, 40, 1))
+    want = torch_softmax_attention(q, k, v, n, 0.25)
+    zero = np.zeros_like(r)
+    for form, got in all_forms(orc, q, zero, k, v, n, 0.25).items():
+        close(got, want, 1e-12, f"r=0 ({form})")
+    close(orc.softmax_decode(q, k, v, n, 0.25), want, 1e-12, "softmax_decode")
+
+
+# ---------------------------------------------------------- closed forms ----
+
+def pin_single_key_returns_v(orc):
+    q, r, k, v, _ = rand_case(2, lengths=(1, 1))
+    want = np.repeat(v[:, :, 0, :], 2, axis=1)  # G = 2
+    for form, got in all_forms(orc, q, r, k, v, [1, 1], 0.3).items():
+        close(got, want, 1e-12, f"single key ({form})")
+
+
+def pin_constant_values(orc):
+    q, r, k, v, n = rand_case(3)
+    c = np.random.default_rng(30).standard_normal((2, 2, 1, 8))
+    v = np.broadcast_to(c, v.shape).copy()
+    want = np.repeat(c[:, :, 0, :], 2, axis=1)
+    for form, got in all_forms(orc, q, r, k, v, n, 0.3).items():
+        close(got, want, 1e-12, f"constant V ({form})")
+
+
+def pin_value_shift_and_scale(orc):
+    q, r, k, v, n = rand_case(4)
+    base = orc.parallax_covariance(q, r, k, v, n, 0.3)
+    c = np.random.default_rng(40).standard_normal(8)
+    for form in FORMS:
+        close(run_form(orc, form, q, r, k, v + c, n, 0.3), base + c, 1e-11,
+              f"V + c ({form})")
+        close(run_form(orc, form, q, r, k, -2.5 * v, n, 0.3), -2.5 * base, 1e-11,
+              f"alpha V ({form})")
+
+
+# ------------------------------------------------------------ invariants ----
+
+def pin_key_translation(orc):
+    """k_i -> k_i + u adds q.u to every logit and r.u to every probe score;
+    neither changes o. A large u also exercises the max subtraction."""
+    q, r, k, v, n = rand_case(5)
+    base = orc.parallax_covariance(q, r, k, v, n, 0.3)
+    u = 40.0 * np.random.default_rng(50).standard_normal(8)
+    for form in FORMS:
+        close(run_form(orc, form, q, r, k + u, v, n, 0.3), base, 1e-9,
+              f"k + u ({form})")
+
+
+def pin_linear_in_r(orc):
+    q, r1, k, v, n = rand_case(6)
+    r2 = np.random.default_rng(60).standard_normal(r1.shape)
+    for form in FORMS:
+        f = lambda r: run_form(orc, form, q, r, k, v, n, 0.3)
+        o0, o1, o2 = f(np.zeros_like(r1)), f(r1), f(r2)
+        close(f(r1 + r2) - o0, (o1 - o0) + (o2 - o0), 1e-10, f"additive in r ({form})")
+        close(f(-3.0 * r1) - o0, -3.0 * (o1 - o0), 1e-10, f"homogeneous in r ({form})")
+        # the correction is not identically zero
+        assert np.max(np.abs(o1 - o0)) > 1e-3, f"r has no effect ({form})"
+
+
+def pin_key_permutation(orc):
+    q, r, k, v, n = rand_case(7, lengths=(24, 24))
+    perm = np.random.default_rng(70).permutation(24)
+    base = orc.parallax_covariance(q, r, k, v, n, 0.3)
+    for form in FORMS:
+        close(run_form(orc, form, q, r, k[:, :, perm], v[:, :, perm], n, 0.3), base,
+              1e-11, f"key permutation ({form})")
+
+
+def pin_forms_agree(orc):
+    """Brute force: definition, expansion and chunked streaming agree."""
+    q, r, k, v, n = rand_case(8, B=4, Hq=8, Hkv=2, D=16, Lmax=70, lengths=(70, 1, 33, 64))
+    base = orc.parallax_covariance(q, r, k, v, n, 0.25)
+    close(orc.parallax_expanded(q, r, k, v, n, 0.25), base, 1e-11, "expanded")
+    for chunk in (1, 2, 5, 16, 64, 70, 1000):
+        close(orc.parallax_streaming(q, r, k, v, n, 0.25, chunk), base, 1e-11,
+              f"streaming chunk={chunk}")
+
+
+# ------------------------------------------- local linear (LLA) intercept ----
+
+def pin_local_linear_intercept(orc):
+    """With r = Sigma_w^{-1}(q - kbar) (LLA's solver output) the Parallax
+    output is the intercept at q of the weighted least-squares fit
+    v_i ~ a + M (k_i - q), weights w_i = softmax(scale q.k_i)."""
+    rng = np.random.default_rng(9)
+    D, n, scale = 4, 15, 0.7
+    q = rng.standard_normal(D)
+    k = rng.standard_normal((n, D))
+    v = rng.standard_normal((n, D))
+    t = scale * k @ q
+    w = np.exp(t - t.max())
+    w /= w.sum()
+    kbar = w @ k
+    sigma = (k - kbar).T @ ((k - kbar) * w[:, None])
+    r = np.linalg.solve(sigma, q - kbar)
+    # weighted least squares with an intercept column
+    X = np.hstack([np.ones((n, 1)), k - q])
+    sw = np.sqrt(w)[:, None]
+    coef, *_ = np.linalg.lstsq(X * sw, v * sw, rcond=None)
+    intercept = coef[0]
+    for form, got in all_forms(orc, q[None, None], r[None, None], k[None, None],
+                               v[None, None], [n], scale).items():
+        close(got[0, 0], intercept, 1e-9, f"LLA intercept ({form})")
+
+
+# ----------------------------------------------- layout, GQA and lengths ----
+
+def pin_gqa_mapping(orc):
+    """Query head h reads kv head h // (Hq/Hkv): give kv head g values g+1."""
+    for Hq, Hkv in ((8, 2), (8, 8), (8, 1), (12, 3)):
+        q, r, k, v, n = rand_case(10, Hq=Hq, Hkv=Hkv)
+        v = np.zeros_like(v)
+        for g in range(Hkv):
+            v[:, g] = g + 1.0
+        want = np.zeros((2, Hq, 8))
+        for h in range(Hq):
+            want[:, h, :] = h // (Hq // Hkv) + 1.0
+        for form, got in all_forms(orc, q, r, k, v, n, 0.3).items():
+            close(got, want, 1e-12, f"GQA {Hq}/{Hkv} ({form})")
+
+
+def pin_lengths_exact(orc):
+    """q = 0 (equal weights), r = 0, value of key i = i: o = (n-1)/2 exactly
+    when exactly keys 0..n-1 are read. NaN padding must not leak."""
+    lengths = (1, 2, 7, 24)
+    q, r, k, v, n = rand_case(11, B=4, lengths=lengths)
+    q[:] = 0.0
+    r[:] = 0.0
+    for i in range(24):
+        v[:, :, i, :] = float(i)
+    for b, nb in enumerate(lengths):
+        k[b, :, nb:, :] = np.nan
+        v[b, :, nb:, :] = np.nan
+    want = np.zeros((4, 4, 8))
+    for b, nb in enumerate(lengths):
+        want[b] = (nb - 1) / 2.0
+    for form, got in all_forms(orc, q, r, k, v, n, 0.3).items():
+        close(got, want, 1e-12, f"lengths ({form})")
+    close(orc.softmax_decode(q, k, v, n, 0.3), want, 1e-12, "lengths (softmax)")
+
+
+def pin_empty_sequence_is_zero(orc):
+    q, r, k, v, _ = rand_case(12)
+    n = [0, 5]
+    k[0] = np.nan
+    v[0] = np.nan
+    for form, got in all_forms(orc, q, r, k, v, n, 0.3).items():
+        assert np.all(got[0] == 0.0), f"empty sequence ({form})"
+        assert np.all(np.isfinite(got[1])), f"finite ({form})"
+
+
+PINS = [pin_hand_examples, pin_r_zero_is_softmax, pin_single_key_returns_v,
+        pin_constant_values, pin_value_shift_and_scale, pin_key_translation,
+        pin_linear_in_r, pin_key_permutation, pin_forms_agree,
+        pin_local_linear_intercept, pin_gqa_mapping, pin_lengths_exact,
+        pin_empty_sequence_is_zero]
