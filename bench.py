@@ -1,0 +1,466 @@
+#!/usr/bin/env python
+"""Parallax decode benchmark on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload qwen|large|long|ragged|tiny]
+    python bench.py --impl reference ...   # the fp64 CPU oracle as the reference arm
+
+A step is one Parallax decode pass (split-KV kernel + merge kernel) over one
+batch of synthetic input resident in HBM. The headline value is KV-read
+bandwidth (algorithmic K and V bytes of the valid keys per step / step time),
+reported next to microseconds per step and the in-run R = 0 softmax decode on
+the same pipeline and buffers. Multi-GPU runs are independent replicas (the
+decode has no cross-GPU exchange), one process per GPU under torchrun.
+
+Timing: CUDA events on the launching stream after W untimed steps, barrier +
+synchronize on both sides, max over ranks. Workloads smaller than the L2
+rotate over enough K/V copies to exceed twice the L2, so every step reads HBM.
+Small workloads are replayed from CUDA graphs (the pages' bench replays
+graphs too: parallax-kernel 0.1.0 README, "Benchmark").
+"""
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from parameterized_local_linear_b200 import inputs  # noqa: E402
+
+METRIC = "decode µs/step and KV-read GB/s (% of HBM peak) vs in-run R=0 softmax decode"
+FALLBACK_HBM_GBS = 6650.0
+DEFAULT_STEPS = {"tiny": 20000, "qwen": 100000, "large": 200, "long": 200, "ragged": 200}
+DEFAULT_WARMUP = {"tiny": 2000, "qwen": 5000, "large": 5, "long": 5, "ragged": 5}
+MAIN_KERNEL_SRC = os.path.join(ROOT, "parameterized_local_linear_b200", "csrc", "kernel_tc.cuh")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=None)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(inputs.WORKLOADS), default="qwen")
+    ap.add_argument("--num-splits", type=int, default=0)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="bound of the CPU oracle baseline sample (seconds)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    a = ap.parse_args()
+    a.steps = a.steps if a.steps is not None else DEFAULT_STEPS[a.workload]
+    a.warmup = a.warmup if a.warmup is not None else DEFAULT_WARMUP[a.workload]
+    return a
+
+
+# ------------------------------------------------------------------ helpers --
+
+def kv_bytes(x) -> int:
+    """Algorithmic K+V bytes of one step: 2 tensors x valid keys x Hkv x D x itemsize."""
+    n = int(x["seqlens"].to(torch.int64).clamp(0, x["k"].shape[2]).sum())
+    _, Hkv, _, D = x["k"].shape
+    return 2 * n * Hkv * D * x["k"].element_size()
+
+
+def qro_bytes(x) -> int:
+    """q and r reads plus the bf16 output write of one step."""
+    return 3 * x["q"].numel() * x["q"].element_size()
+
+
+def workload_desc(w: inputs.Workload) -> str:
+    lens = {"full": f"L={w.Lmax}", "uniform": f"L~U[1,{w.Lmax}]"}.get(
+        w.lengths if isinstance(w.lengths, str) else "", f"L={list(w.lengths)}")
+    return (f"{w.name}: Parallax decode B={w.B} Hq={w.Hq} Hkv={w.Hkv} D={w.D} {lens} "
+            f"Lmax={w.Lmax} {str(w.dtype).replace('torch.', '')}")
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def profiled_traffic():
+    """Per-launch DRAM traffic of the split-KV kernel from the committed ncu
+    summary, if it was taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "parallax_tc_kernel_qwen.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    src_hash = hashlib.sha256(open(MAIN_KERNEL_SRC, "rb").read()).hexdigest()[:16]
+    m_hash = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
+    m_traffic = re.search(r"traffic_bytes_per_launch:\s*([0-9]+)", text)
+    if not m_hash or not m_traffic or m_hash.group(1) != src_hash:
+        return None
+    return int(m_traffic.group(1))
+
+
+class ClockSampler:
+    """Samples SM clock, power and clock-event reasons through NVML while the
+    timed region runs (reads only; changes no setting)."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.02):
+        self.samples, self.period, self._stop = [], period_s, threading.Event()
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            uuid = torch.cuda.get_device_properties(device_index).uuid
+            self.h = None
+            for i in range(pynvml.nvmlDeviceGetCount()):
+                h = pynvml.nvmlDeviceGetHandleByIndex(i)
+                u = pynvml.nvmlDeviceGetUUID(h)
+                u = u.decode() if isinstance(u, bytes) else u
+                if str(uuid) in u:
+                    self.h = h
+            if self.h is None:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report that, do not guess
+            self.err = repr(e)
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((mhz, reasons))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "error": getattr(self, "err", "nvml unavailable")}
+        mhz = [s[0] for s in self.samples]
+        bits = 0
+        for _, r in self.samples:
+            bits |= int(r)
+        reasons = sorted(v for k, v in self.REASONS.items() if bits & k)
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(mhz)}
+
+
+class Dist:
+    def __init__(self, gpus: int):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        if gpus != self.world:
+            raise SystemExit(f"--gpus {gpus} but WORLD_SIZE={self.world}: launch N>1 with torchrun")
+        self.pg = None
+
+    def init_gpu(self):
+        torch.cuda.set_device(self.local)
+        if self.world > 1:
+            import torch.distributed as dist
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                    device_id=torch.device("cuda", self.local))
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg:
+            self.pg.barrier()
+
+    def max(self, x: float) -> float:
+        if not self.pg:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            self.pg.destroy_process_group()
+
+
+# ------------------------------------------------------------ CPU oracle ----
+
+def oracle_sample(w: inputs.Workload, x_host: dict, budget_s: float):
+    """Time the fp64 oracle, as it stands, on a bounded sample of the workload.
+    Returns (GB/s of KV processed, cores, description, seconds)."""
+    import oracle
+    rows_all = list(range(w.B))
+    lens = x_host["seqlens"].tolist()
+    per_row = [2 * n * w.Hkv * w.D * x_host["k"].element_size() for n in lens]
+    # grow the sample one batch row at a time until its first pass is ~1/5 of the budget
+    done_bytes, elapsed, rows, reps = 0, 0.0, [], 0
+    t_start = time.perf_counter()
+    order = rows_all
+    i = 0
+    while elapsed < budget_s:
+        if i < len(order) and (not rows or elapsed < budget_s / 5):
+            rows.append(order[i])
+            i += 1
+            sel = rows[-1:]
+        else:
+            sel = rows
+            reps += 1
+        idx = torch.tensor(sel)
+        t0 = time.perf_counter()
+        oracle.parallax_decode(x_host["q"][idx], x_host["r"][idx], x_host["k"][idx],
+                               x_host["v"][idx], x_host["seqlens"][idx], x_host["scale"])
+        elapsed += time.perf_counter() - t0
+        done_bytes += sum(per_row[b] for b in sel)
+        if time.perf_counter() - t_start > 3 * budget_s:
+            break
+    desc = (f"fp64 oracle (covariance form) on batch rows {rows[0]}..{rows[-1]} "
+            f"({len(rows)} of {w.B} rows, {reps} extra passes); {elapsed:.1f} s")
+    return done_bytes / elapsed / 1e9, oracle.num_threads(), desc, elapsed
+
+
+def host_inputs_for_oracle(w: inputs.Workload, budget_rows: int = 64):
+    """The workload's seeded inputs on the host, limited to the first rows the
+    oracle can take (large workloads are drawn on the GPU and copied back)."""
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    x = inputs.make_inputs(w, device=dev, pad_value=None)
+    rows = min(w.B, budget_rows)
+    out = {k: (v[:rows].cpu() if torch.is_tensor(v) else v) for k, v in x.items()}
+    del x
+    if dev == "cuda":
+        torch.cuda.empty_cache()
+    wsub = inputs.Workload(w.name, rows, w.Hq, w.Hkv, w.D, w.Lmax, w.dtype, w.seed, "full",
+                           w.r_scale, w.k_offset_std, w.scale)
+    return wsub, out
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = inputs.WORKLOADS[args.workload]
+    wsub, xh = host_inputs_for_oracle(w)
+    per_step_budget = max(1.0, 120.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        oracle_sample(wsub, xh, min(per_step_budget, 2.0))
+    vals, secs, desc, cores = [], 0.0, "", 0
+    for _ in range(args.steps):
+        v, cores, desc, s = oracle_sample(wsub, xh, per_step_budget)
+        vals.append(v)
+        secs += s
+    value = statistics.median(vals)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": secs / max(1, args.steps) * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": workload_desc(w), "parallelism": "rank 0 only (host CPU)"},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+# ------------------------------------------------------------- GPU timing ----
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    from parameterized_local_linear_b200 import binding
+
+    dist = Dist(args.gpus)
+    dist.init_gpu()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    binding.load_library()
+    w = inputs.WORKLOADS[args.workload]
+    stream = torch.cuda.Stream(device=dev)  # graphs can not be captured on the legacy stream
+    torch.cuda.set_stream(stream)
+
+    x = inputs.make_inputs(w, device=dev, pad_value=None)
+    step_kv = kv_bytes(x)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    nbuf = 1
+    if w.kv_bytes_full() < 2 * l2:
+        nbuf = max(2, math.ceil(2 * l2 / w.kv_bytes_full()))
+        l2_note = f"rotate {nbuf} K/V copies ({nbuf * w.kv_bytes_full() / 1e6:.0f} MB > 2x L2)"
+    else:
+        l2_note = f"inputs ({w.kv_bytes_full() / 1e9:.1f} GB of K/V) larger than L2"
+    bufs = [x] + [{k: (v.clone() if torch.is_tensor(v) else v) for k, v in x.items()}
+                  for _ in range(nbuf - 1)]
+    out = torch.empty((w.B, w.Hq, w.D), device=dev, dtype=torch.bfloat16)
+    P = args.num_splits if args.num_splits > 0 else binding.parallax_choose_splits(w.B, w.Hkv, w.Lmax)
+    ws = binding.Workspace(w.B, w.Hq, w.Hkv, w.D, w.Lmax, P, device=dev)
+
+    def step(b, probe=True):
+        if probe:
+            binding.parallax_decode(b["q"], b["r"], b["k"], b["v"], b["seqlens"], scale=b["scale"],
+                                    out=out, num_splits=P, workspace=ws, stream=stream)
+        else:
+            binding.parallax_softmax_decode(b["q"], b["k"], b["v"], b["seqlens"],
+                                            scale=b["scale"], out=out, num_splits=P,
+                                            workspace=ws, stream=stream)
+
+    use_graphs = nbuf > 1
+
+    def make_runner(probe):
+        if not use_graphs:
+            def run(k):
+                for i in range(k):
+                    step(bufs[i % nbuf], probe)
+            return run
+        for b in bufs:  # warm the launch path outside capture
+            step(b, probe)
+        torch.cuda.synchronize()
+        chain = torch.cuda.CUDAGraph()
+        singles = []
+        with torch.cuda.graph(chain, stream=stream):
+            for b in bufs:
+                step(b, probe)
+        for b in bufs:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                step(b, probe)
+            singles.append(g)
+
+        def run(k):
+            for _ in range(k // nbuf):
+                chain.replay()
+            for i in range(k % nbuf):
+                singles[i].replay()
+        return run
+
+    def timed(run, k, w_steps, sampler=None):
+        run(w_steps)
+        torch.cuda.synchronize()
+        dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if sampler:
+            sampler.__enter__()
+        e0.record(stream)
+        run(k)
+        e1.record(stream)
+        e1.synchronize()
+        if sampler:
+            sampler.__exit__(None, None, None)
+        torch.cuda.synchronize()
+        dist.barrier()
+        return dist.max(e0.elapsed_time(e1) / 1e3)
+
+    run_plx = make_runner(True)
+    run_soft = make_runner(False)
+    sampler = ClockSampler(dev.index)
+    t_plx = timed(run_plx, args.steps, args.warmup, sampler)
+    t_soft = timed(run_soft, args.steps, args.warmup)
+    rc, bits = ws.status()
+    if rc != 0:
+        raise SystemExit(f"device status after timing: {binding.parallax_status_string(rc)}")
+
+    # ---- per-kernel duration of the split-KV kernel (phase 1), live ----
+    nprof = min(args.steps, 1000 if use_graphs else 50)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(nprof)]
+    for i in range(3):
+        step(bufs[i % nbuf])
+    torch.cuda.synchronize()
+    torch.cuda._sleep(int(4e8))  # let the host queue the launches ahead of the GPU
+    for i, (a, b) in enumerate(evs):
+        bb = bufs[i % nbuf]
+        a.record(stream)
+        binding.parallax_decode_phase(1, True, bb["q"], bb["r"], bb["k"], bb["v"], bb["seqlens"],
+                                      out, ws, scale=bb["scale"], num_splits=P, stream=stream)
+        b.record(stream)
+        binding.parallax_decode_phase(2, True, bb["q"], bb["r"], bb["k"], bb["v"], bb["seqlens"],
+                                      out, ws, scale=bb["scale"], num_splits=P, stream=stream)
+    torch.cuda.synchronize()
+    main_s = statistics.mean(a.elapsed_time(b) for a, b in evs) / 1e3
+
+    # ---- end to end through the public API with host buffers ----
+    pin = {k: x[k].cpu().pin_memory() for k in ("q", "r", "seqlens")}
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    k_e2e = min(args.steps, 2000 if use_graphs else args.steps)
+
+    def run_e2e(k):
+        for i in range(k):
+            b = bufs[i % nbuf]
+            b["q"].copy_(pin["q"], non_blocking=True)
+            b["r"].copy_(pin["r"], non_blocking=True)
+            b["seqlens"].copy_(pin["seqlens"], non_blocking=True)
+            step(b)
+            out_host.copy_(out, non_blocking=True)
+
+    t_e2e = timed(run_e2e, k_e2e, min(args.warmup, 50))
+    h2d = sum(pin[k].numel() * pin[k].element_size() for k in pin)
+    d2h = out_host.numel() * out_host.element_size()
+
+    # ---- CPU oracle baseline (rank 0, N = 1 only) ----
+    cpu = None
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        xh = {k: (v[: min(w.B, 64)].cpu() if torch.is_tensor(v) else v) for k, v in x.items()}
+        wsub = inputs.Workload(w.name, min(w.B, 64), w.Hq, w.Hkv, w.D, w.Lmax, w.dtype, w.seed,
+                               "full", w.r_scale, w.k_offset_std, w.scale)
+        xh["seqlens"] = x["seqlens"][: wsub.B].cpu()
+        v, cores, desc, _ = oracle_sample(wsub, xh, args.cpu_seconds)
+        cpu = {"value": v, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": desc}
+
+    hbm_peak, peak_src = measured_peaks()
+    N = dist.world
+    gbs = N * args.steps * step_kv / t_plx / 1e9
+    main_bytes = step_kv + qro_bytes(x)
+    achieved = main_bytes / main_s / 1e9
+    clocks = sampler.summary()
+    line = {
+        "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": N, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": t_plx / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": workload_desc(w), "global_batch": w.B * N, "seq_len": w.Lmax,
+                   "parallelism": f"replicas x{N}" if N > 1 else "single GPU",
+                   "num_splits": P, "l2": l2_note, "cuda_graphs": use_graphs},
+        "us_per_step": t_plx / args.steps * 1e6,
+        "kv_gbs_frac_of_hbm_peak": gbs / N / hbm_peak,
+        "softmax_r0": {"us_per_step": t_soft / args.steps * 1e6,
+                       "kv_gbs": N * args.steps * step_kv / t_soft / 1e9,
+                       "parallax_over_softmax_latency": t_plx / t_soft},
+        "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons", "samples")},
+        "e2e": {"value": N * k_e2e * step_kv / t_e2e / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "us_per_step": t_e2e / k_e2e * 1e6},
+        "gpu_launches": 2 * args.steps,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved / hbm_peak, "traffic": profiled_traffic(),
+                     "kernel": "parallax_tc_kernel (split-KV)", "peak_source": peak_src,
+                     "kernel_us": main_s * 1e6, "algorithmic_bytes_per_launch": main_bytes},
+        "cpu_baseline": cpu,
+    }
+    if dist.rank == 0:
+        print(json.dumps(line))
+    dist.close()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,167 @@
+/*
+ * parallax.h - C ABI of libparallax.so, the B200 (sm_100a) Parallax decode.
+ *
+ * Parallax (parameterized Local Linear Attention) keeps softmax attention's
+ * readout and adds a learned covariance correction: each query head carries
+ * its query q and a probe r produced by a learned projector, and the decode
+ * output over the cached keys k_i and values v_i is
+ *
+ *     w_i = softmax_i(scale * q.k_i),   s_i = r.k_i,
+ *     o   = vbar + sum_i w_i (s_i - sbar)(v_i - vbar)
+ *         = A/l + C/l - (b/l)(A/l),
+ *     l = sum e_i, A = sum e_i v_i, b = sum e_i s_i, C = sum e_i s_i v_i,
+ *     e_i = exp(scale * q.k_i - m).
+ *
+ * Sources: "Parallax: Parameterized Local Linear Attention for Language
+ * Modeling" (neuraltrendhub summary, "What the paper found" and "Original
+ * abstract": the learned query-like projector that probes the KV covariance
+ * in place of LLA's solve, one streaming pass over FlashAttention's K/V
+ * tiles); same title (bayesiansapien blog, opening diagram and "TL;DR":
+ * softmax is the local-constant estimate, LLA the local-linear one);
+ * parallax-kernel 0.1.0 README, "Decoding (CuTeDSL)": the decode call takes
+ * q, r (shaped like q), k, v and qk_scale; "Integrazioni AI personalizzate
+ * dopo l'attenzione Parallax" (encorp.ai), FAQ: with the projection at zero
+ * the layer is exactly softmax attention.
+ *
+ * Conventions shared by every entry point
+ * ----------------------------------------
+ *  - All tensor pointers are DEVICE pointers owned by the caller. The library
+ *    allocates no device memory and keeps no per-call state; the workspace is
+ *    caller-owned scratch (see parallax_decode_workspace_bytes).
+ *  - Layouts are contiguous, row-major, innermost last:
+ *        q, r, out      [B][Hq][D]
+ *        k_cache,v_cache[B][Hkv][Lmax][D]     (max-length-padded cache)
+ *        cache_seqlens  [B] int32             (device memory)
+ *    Query head h reads kv head h / (Hq/Hkv) (contiguous GQA groups). Keys
+ *    0 .. cache_seqlens[b]-1 of sequence b are attended; padding positions
+ *    are never read into any accumulator. Values outside [0, Lmax] are
+ *    clamped on the device and reported through the workspace status word.
+ *    A sequence with no keys gets a zero output.
+ *  - in_dtype: PARALLAX_DTYPE_BF16 or PARALLAX_DTYPE_F32 (q, r, k, v alike).
+ *    out_dtype: PARALLAX_DTYPE_BF16 (round-to-nearest-even from fp32) or
+ *    PARALLAX_DTYPE_F32 (the fp32 debug output). Accumulation is fp32.
+ *  - D must be 64 or 128. Hq must be a multiple of Hkv. All pointers must be
+ *    16-byte aligned.
+ *  - scale is the softmax scale applied to q.k only (qk_scale); the probe
+ *    score s_i = r.k_i is not scaled.
+ *  - stream is a cudaStream_t (NULL = legacy default stream). Calls are
+ *    stream-ordered and asynchronous: no host synchronisation, no allocation,
+ *    so they can be captured in a CUDA graph.
+ *  - num_splits: 0 lets parallax_choose_splits pick the number of key-range
+ *    partitions for the device; a positive value forces it (1 .. 65536).
+ *    Results do not depend on it beyond fp32 rounding, and are bitwise
+ *    reproducible for a fixed value and device.
+ *  - Return value: PARALLAX_OK (0) or a negative status. Argument errors are
+ *    detected on the host before anything is launched. Launch failures return
+ *    PARALLAX_ERR_CUDA. Nothing is thrown across the ABI.
+ */
+#ifndef PARALLAX_H
+#define PARALLAX_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define PARALLAX_OK 0
+#define PARALLAX_ERR_NULL_POINTER (-1)
+#define PARALLAX_ERR_BAD_SHAPE (-2)
+#define PARALLAX_ERR_UNSUPPORTED_HEAD_DIM (-3)
+#define PARALLAX_ERR_UNSUPPORTED_DTYPE (-4)
+#define PARALLAX_ERR_MISALIGNED (-5)
+#define PARALLAX_ERR_WORKSPACE_TOO_SMALL (-6)
+#define PARALLAX_ERR_BAD_SPLITS (-7)
+#define PARALLAX_ERR_CUDA (-8)
+#define PARALLAX_ERR_DEVICE_TIMEOUT (-9)
+#define PARALLAX_ERR_BAD_PHASE (-10)
+#define PARALLAX_ERR_SEQLEN_CLAMPED (-11)
+
+#define PARALLAX_DTYPE_BF16 0
+#define PARALLAX_DTYPE_F32 1
+
+#define PARALLAX_MAX_SPLITS 65536
+
+/* Bits of the device status word kept at the start of the workspace. */
+#define PARALLAX_DEVICE_STATUS_TIMEOUT 1u
+#define PARALLAX_DEVICE_STATUS_SEQLEN_CLAMPED 2u
+
+/*
+ * Number of key-range partitions (CTAs of the persistent split-KV kernel) the
+ * library uses by default: the flattened (batch, kv head, key) range is cut
+ * into this many equal parts, so a number of whole waves of the device's SMs
+ * is kept busy whatever the batch size and lengths. sm_count <= 0 queries the
+ * current device. Returns >= 1, or a negative status for bad arguments.
+ */
+int parallax_choose_splits(int B, int Hkv, int Lmax, int sm_count);
+
+/*
+ * Bytes of workspace one decode call needs: a 256-byte header (the device
+ * status word) plus two fp32 partial records (m, l, b, A[D], C[D]) per
+ * partition and query head of a group. num_splits as in parallax_decode (0 =
+ * the default for the current device). Returns 0 for invalid arguments.
+ * The workspace must be zero-filled once after allocation (the status word);
+ * the partial records need no initialisation.
+ */
+size_t parallax_decode_workspace_bytes(int B, int Hq, int Hkv, int D, int Lmax,
+                                       int num_splits);
+
+/*
+ * The Parallax decode forward: out = vbar + C/l - (b/l) vbar per query head
+ * (see the top of this file). r holds the probe rows, one per query head,
+ * shaped like q. Launches the split-KV kernel and the split-merge kernel on
+ * `stream`.
+ */
+int parallax_decode(const void* q, const void* r, const void* k_cache,
+                    const void* v_cache, const int32_t* cache_seqlens, void* out,
+                    int B, int Hq, int Hkv, int D, float scale, void* stream,
+                    int Lmax, int in_dtype, int out_dtype, int num_splits,
+                    void* workspace, size_t workspace_bytes);
+
+/*
+ * The R = 0 comparator: plain softmax attention decode (out = A/l), the
+ * FlashAttention-style kernel Parallax reduces to when the probe projection
+ * is zero. Same pipeline and arguments as parallax_decode, without r.
+ */
+int parallax_softmax_decode(const void* q, const void* k_cache,
+                            const void* v_cache, const int32_t* cache_seqlens,
+                            void* out, int B, int Hq, int Hkv, int D, float scale,
+                            void* stream, int Lmax, int in_dtype, int out_dtype,
+                            int num_splits, void* workspace,
+                            size_t workspace_bytes);
+
+/*
+ * One phase of a decode call, for per-kernel timing and for tests of the
+ * partial records: phase 1 runs only the split-KV kernel (writes `out` for
+ * sequences covered by one partition and partial records for the others),
+ * phase 2 only the split-merge kernel. Calling phase 1 then phase 2 with the
+ * same arguments is equivalent to one call of parallax_decode (probe = 1) or
+ * parallax_softmax_decode (probe = 0; r may be NULL). Returns
+ * PARALLAX_ERR_BAD_PHASE for any other phase.
+ */
+int parallax_decode_phase(int phase, int probe, const void* q, const void* r,
+                          const void* k_cache, const void* v_cache,
+                          const int32_t* cache_seqlens, void* out, int B, int Hq,
+                          int Hkv, int D, float scale, void* stream, int Lmax,
+                          int in_dtype, int out_dtype, int num_splits,
+                          void* workspace, size_t workspace_bytes);
+
+/*
+ * Synchronise the current device, then read (and, if clear != 0, zero) the
+ * device status word at the start of a workspace. *device_status receives PARALLAX_DEVICE_STATUS_* bits;
+ * the return value maps them to a status: PARALLAX_ERR_DEVICE_TIMEOUT if a
+ * bounded wait inside a kernel gave up (the kernel then returned early and its
+ * output is invalid), PARALLAX_ERR_SEQLEN_CLAMPED if a length was outside
+ * [0, Lmax], else PARALLAX_OK.
+ */
+int parallax_workspace_status(void* workspace, int clear, uint32_t* device_status);
+
+/* Human-readable text for a status code; never NULL. */
+const char* parallax_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PARALLAX_H */

@@ -1,0 +1,70 @@
+// Definitions shared by the host launcher and the kernels.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+namespace plx {
+
+// Workspace: a 256-byte header whose first word is the device status word,
+// then 2 * P * G partial records of kRecHead + 2*D floats each:
+//   [0] m (running max, log2 domain) [1] l [2] b [3] unused [4..4+D) A [4+D..4+2D) C
+constexpr size_t kWorkspaceHeaderBytes = 256;
+constexpr int kRecHead = 4;
+
+__host__ __device__ constexpr int rec_floats(int D) { return kRecHead + 2 * D; }
+
+struct DecodeParams {
+  const void* q;          // [B][Hq][D]
+  const void* r;          // [B][Hq][D] (unused by the softmax kernels)
+  const void* k;          // [B][Hkv][Lmax][D] (generic kernel only; the TMA kernel uses tensor maps)
+  const void* v;
+  const int32_t* seqlens; // [B]
+  void* out;              // [B][Hq][D]
+  float* partials;        // 2 * P * G records
+  unsigned int* status;   // device status word (workspace header)
+  int B, Hq, Hkv, G, D, Lmax;
+  float scale_log2;       // qk_scale * log2(e): logits are kept in the log2 domain
+  unsigned long long timeout_ns;  // bound of every wait inside the kernels
+  int debug_skip_first_tile;      // testing hook: the producer never fills stage 0
+};
+
+// ------------------------------------------------ TMA kernel geometry ------
+constexpr int kTileKeys = 64;        // keys per pipeline stage
+constexpr int kConsumerWarps = 4;    // each owns 16 keys of a stage
+constexpr int kTcThreads = (kConsumerWarps + 1) * 32;  // + one producer warp
+constexpr int kBoxBytes = kTileKeys * 128;             // one 64-key x 128-byte swizzled box
+
+template <int D>
+struct TcGeom {
+  static constexpr int kHalves = D / 64;                 // 128-byte boxes per key row
+  static constexpr int kKBytes = kHalves * kBoxBytes;    // K tile of one stage
+  static constexpr int kStageBytes = 2 * kKBytes;        // K + V
+  static constexpr int kStages = D == 128 ? 3 : 6;       // 96 KB of ring either way
+};
+
+__host__ __device__ constexpr int align_up(int x, int a) { return (x + a - 1) / a * a; }
+
+// Byte offsets inside the (1024-aligned) dynamic shared memory of the TMA kernel.
+struct TcSmemLayout {
+  int qr_slot_bytes, off_qr, off_p, off_merge, off_bar, off_misc, total;
+};
+
+__host__ __device__ inline TcSmemLayout tc_smem_layout(int D, int stage_bytes, int stages, int G,
+                                                       bool probe) {
+  TcSmemLayout L{};
+  L.qr_slot_bytes = align_up((probe ? 2 : 1) * G * D * 2, 128);
+  L.off_qr = stages * stage_bytes;
+  L.off_p = L.off_qr + 2 * L.qr_slot_bytes;
+  L.off_merge = L.off_p + kConsumerWarps * 512;
+  L.off_bar = align_up(L.off_merge + kConsumerWarps * G * rec_floats(D) * 4, 16);
+  // full[stages], empty[stages], qr_full[2], qr_empty[2], fin[2]
+  L.off_misc = L.off_bar + 8 * (2 * stages + 6);
+  L.total = L.off_misc + 512 + 1024;  // prologue scratch, abort flag, alignment slack
+  return L;
+}
+
+constexpr int kGenericThreads = 128;
+constexpr int kMergeThreads = 128;
+
+}  // namespace plx

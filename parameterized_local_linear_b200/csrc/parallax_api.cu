@@ -1,0 +1,363 @@
+// C ABI of libparallax.so (declared in include/parallax.h): argument checks,
+// the split-count heuristic, TMA descriptor encoding and kernel launches.
+// The host never synchronises and never allocates; every launch goes to the
+// caller's stream.
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "parallax.h"
+
+#include "common.cuh"
+#include "kernel_generic.cuh"
+#include "kernel_merge.cuh"
+#include "kernel_tc.cuh"
+
+using namespace plx;
+
+namespace {
+
+constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;  // 2 s per wait
+constexpr long long kMinKeysPerSplit = 64;  // smallest key range worth a CTA
+constexpr int kCtasPerSm = 2;               // split-KV CTAs resident per SM
+
+struct Call {
+  int phases;  // bit 0: split-KV kernel, bit 1: merge kernel
+  bool probe;
+  const void *q, *r, *k, *v;
+  const int32_t* seqlens;
+  void* out;
+  int B, Hq, Hkv, D;
+  float scale;
+  cudaStream_t stream;
+  int Lmax, in_dtype, out_dtype, num_splits;
+  void* ws;
+  size_t ws_bytes;
+  unsigned long long timeout_ns;
+  int debug_skip_first_tile;
+};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int current_sm_count(int* out) {
+  static int cache[256] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PARALLAX_ERR_CUDA;
+  if (dev >= 0 && dev < 256 && cache[dev] > 0) {
+    *out = cache[dev];
+    return PARALLAX_OK;
+  }
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
+    return PARALLAX_ERR_CUDA;
+  if (dev >= 0 && dev < 256) cache[dev] = n;
+  *out = n;
+  return PARALLAX_OK;
+}
+
+int choose_splits_impl(int B, int Hkv, int Lmax, int sm_count) {
+  const long long max_keys = (long long)B * Hkv * Lmax;
+  const long long slots = (long long)kCtasPerSm * sm_count;
+  const long long by_work = std::max(1LL, (max_keys + kMinKeysPerSplit - 1) / kMinKeysPerSplit);
+  return (int)std::min(slots, by_work);
+}
+
+bool shape_ok(int B, int Hq, int Hkv, int D, int Lmax) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || Lmax < 1 || D < 1) return false;
+  if (Hq % Hkv != 0) return false;
+  if ((long long)B * Hkv > 0x7fffffffLL) return false;  // TMA item coordinate is int32
+  return true;
+}
+
+size_t workspace_bytes_for(int G, int D, int P) {
+  return kWorkspaceHeaderBytes + (size_t)2 * P * G * rec_floats(D) * sizeof(float);
+}
+
+int resolve_splits(int num_splits, int B, int Hkv, int Lmax, int* P) {
+  if (num_splits < 0 || num_splits > PARALLAX_MAX_SPLITS) return PARALLAX_ERR_BAD_SPLITS;
+  if (num_splits > 0) {
+    *P = num_splits;
+    return PARALLAX_OK;
+  }
+  int sm = 0;
+  const int st = current_sm_count(&sm);
+  if (st != PARALLAX_OK) return st;
+  *P = choose_splits_impl(B, Hkv, Lmax, sm);
+  return PARALLAX_OK;
+}
+
+int validate(const Call& c) {
+  if (!c.q || !c.k || !c.v || !c.seqlens || !c.out || !c.ws) return PARALLAX_ERR_NULL_POINTER;
+  if (c.probe && !c.r) return PARALLAX_ERR_NULL_POINTER;
+  if (!shape_ok(c.B, c.Hq, c.Hkv, c.D, c.Lmax)) return PARALLAX_ERR_BAD_SHAPE;
+  if (c.D != 64 && c.D != 128) return PARALLAX_ERR_UNSUPPORTED_HEAD_DIM;
+  if ((c.in_dtype != PARALLAX_DTYPE_BF16 && c.in_dtype != PARALLAX_DTYPE_F32) ||
+      (c.out_dtype != PARALLAX_DTYPE_BF16 && c.out_dtype != PARALLAX_DTYPE_F32))
+    return PARALLAX_ERR_UNSUPPORTED_DTYPE;
+  if (!aligned16(c.q) || (c.probe && !aligned16(c.r)) || !aligned16(c.k) || !aligned16(c.v) ||
+      !aligned16(c.out) || !aligned16(c.ws) || (reinterpret_cast<uintptr_t>(c.seqlens) & 3u))
+    return PARALLAX_ERR_MISALIGNED;
+  if (c.num_splits < 0 || c.num_splits > PARALLAX_MAX_SPLITS) return PARALLAX_ERR_BAD_SPLITS;
+  return PARALLAX_OK;
+}
+
+// --------------------------------------------------------- TMA descriptors --
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// [B*Hkv][Lmax][D] bf16 cache, boxes of 64 keys x 64 dims (128 bytes, swizzled).
+int encode_cache_map(CUtensorMap* map, const void* cache, int D, int Lmax, long long items) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return PARALLAX_ERR_CUDA;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Lmax, (cuuint64_t)items};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)Lmax * D * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)kTileKeys, 1};
+  cuuint32_t elem[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(cache), dims,
+                   strides, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? PARALLAX_OK : PARALLAX_ERR_CUDA;
+}
+
+// ----------------------------------------------------------------- launch --
+
+template <typename Kernel>
+int set_smem_once(Kernel kernel, int bytes, int* done_dev) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PARALLAX_ERR_CUDA;
+  if (dev >= 0 && dev < 256 && done_dev[dev] >= bytes) return PARALLAX_OK;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+      cudaSuccess)
+    return PARALLAX_ERR_CUDA;
+  if (dev >= 0 && dev < 256) done_dev[dev] = bytes;
+  return PARALLAX_OK;
+}
+
+template <int D, bool PROBE, bool OUT_F32>
+int launch_tc(const Call& c, const DecodeParams& prm, int P) {
+  // probabilities as bf16 hi + lo: always with the probe, else for fp32 output
+  constexpr bool kPsplit = PROBE || OUT_F32;
+  auto kernel = parallax_tc_kernel<D, PROBE, OUT_F32, kPsplit>;
+  static int done[256] = {0};
+  const TcSmemLayout L =
+      tc_smem_layout(D, TcGeom<D>::kStageBytes, TcGeom<D>::kStages, prm.G, PROBE);
+  int st = set_smem_once(kernel, L.total, done);
+  if (st != PARALLAX_OK) return st;
+  CUtensorMap tmK, tmV;
+  const long long items = (long long)c.B * c.Hkv;
+  if ((st = encode_cache_map(&tmK, c.k, D, c.Lmax, items)) != PARALLAX_OK) return st;
+  if ((st = encode_cache_map(&tmV, c.v, D, c.Lmax, items)) != PARALLAX_OK) return st;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)P);
+  cfg.blockDim = dim3(kTcThreads);
+  cfg.dynamicSmemBytes = (size_t)L.total;
+  cfg.stream = c.stream;
+  return cudaLaunchKernelEx(&cfg, kernel, tmK, tmV, prm) == cudaSuccess ? PARALLAX_OK
+                                                                        : PARALLAX_ERR_CUDA;
+}
+
+template <typename T, bool PROBE, bool OUT_F32>
+int launch_generic(const Call& c, const DecodeParams& prm, int P) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)P);
+  cfg.blockDim = dim3(kGenericThreads);
+  cfg.stream = c.stream;
+  return cudaLaunchKernelEx(&cfg, parallax_generic_kernel<T, PROBE, OUT_F32>, prm) == cudaSuccess
+             ? PARALLAX_OK
+             : PARALLAX_ERR_CUDA;
+}
+
+template <bool PROBE, bool OUT_F32>
+int launch_merge(const Call& c, const DecodeParams& prm, int P) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)P);
+  cfg.blockDim = dim3(kMergeThreads);
+  cfg.stream = c.stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, parallax_merge_kernel<PROBE, OUT_F32>, prm) == cudaSuccess
+             ? PARALLAX_OK
+             : PARALLAX_ERR_CUDA;
+}
+
+template <bool PROBE, bool OUT_F32>
+int launch_split_kv(const Call& c, const DecodeParams& prm, int P) {
+  const bool tc_ok = c.in_dtype == PARALLAX_DTYPE_BF16 && (PROBE ? 2 * prm.G <= 8 : prm.G <= 8);
+  if (tc_ok) {
+    if (c.D == 128) return launch_tc<128, PROBE, OUT_F32>(c, prm, P);
+    return launch_tc<64, PROBE, OUT_F32>(c, prm, P);
+  }
+  if (c.in_dtype == PARALLAX_DTYPE_BF16) return launch_generic<__nv_bfloat16, PROBE, OUT_F32>(c, prm, P);
+  return launch_generic<float, PROBE, OUT_F32>(c, prm, P);
+}
+
+template <bool PROBE, bool OUT_F32>
+int run_phases(const Call& c, const DecodeParams& prm, int P) {
+  if (c.phases & 1) {
+    const int st = launch_split_kv<PROBE, OUT_F32>(c, prm, P);
+    if (st != PARALLAX_OK) return st;
+  }
+  if (c.phases & 2) return launch_merge<PROBE, OUT_F32>(c, prm, P);
+  return PARALLAX_OK;
+}
+
+int run(const Call& c) {
+  int st = validate(c);
+  if (st != PARALLAX_OK) return st;
+  int P = 0;
+  if ((st = resolve_splits(c.num_splits, c.B, c.Hkv, c.Lmax, &P)) != PARALLAX_OK) return st;
+  const int G = c.Hq / c.Hkv;
+  if (c.ws_bytes < workspace_bytes_for(G, c.D, P)) return PARALLAX_ERR_WORKSPACE_TOO_SMALL;
+
+  DecodeParams prm{};
+  prm.q = c.q;
+  prm.r = c.probe ? c.r : nullptr;
+  prm.k = c.k;
+  prm.v = c.v;
+  prm.seqlens = c.seqlens;
+  prm.out = c.out;
+  prm.status = static_cast<unsigned int*>(c.ws);
+  prm.partials = reinterpret_cast<float*>(static_cast<char*>(c.ws) + kWorkspaceHeaderBytes);
+  prm.B = c.B;
+  prm.Hq = c.Hq;
+  prm.Hkv = c.Hkv;
+  prm.G = G;
+  prm.D = c.D;
+  prm.Lmax = c.Lmax;
+  prm.scale_log2 = (float)((double)c.scale * 1.4426950408889634);  // log2(e)
+  prm.timeout_ns = c.timeout_ns;
+  prm.debug_skip_first_tile = c.debug_skip_first_tile;
+
+  const bool f32 = c.out_dtype == PARALLAX_DTYPE_F32;
+  if (c.probe) return f32 ? run_phases<true, true>(c, prm, P) : run_phases<true, false>(c, prm, P);
+  return f32 ? run_phases<false, true>(c, prm, P) : run_phases<false, false>(c, prm, P);
+}
+
+Call make_call(int phases, bool probe, const void* q, const void* r, const void* k, const void* v,
+               const int32_t* seqlens, void* out, int B, int Hq, int Hkv, int D, float scale,
+               void* stream, int Lmax, int in_dtype, int out_dtype, int num_splits, void* ws,
+               size_t ws_bytes) {
+  Call c;
+  c.phases = phases;
+  c.probe = probe;
+  c.q = q;
+  c.r = r;
+  c.k = k;
+  c.v = v;
+  c.seqlens = seqlens;
+  c.out = out;
+  c.B = B;
+  c.Hq = Hq;
+  c.Hkv = Hkv;
+  c.D = D;
+  c.scale = scale;
+  c.stream = static_cast<cudaStream_t>(stream);
+  c.Lmax = Lmax;
+  c.in_dtype = in_dtype;
+  c.out_dtype = out_dtype;
+  c.num_splits = num_splits;
+  c.ws = ws;
+  c.ws_bytes = ws_bytes;
+  c.timeout_ns = kDefaultTimeoutNs;
+  c.debug_skip_first_tile = 0;
+  return c;
+}
+
+}  // namespace
+
+extern "C" {
+
+int parallax_choose_splits(int B, int Hkv, int Lmax, int sm_count) {
+  if (B < 1 || Hkv < 1 || Lmax < 1) return PARALLAX_ERR_BAD_SHAPE;
+  if (sm_count <= 0) {
+    const int st = current_sm_count(&sm_count);
+    if (st != PARALLAX_OK) return st;
+  }
+  return choose_splits_impl(B, Hkv, Lmax, sm_count);
+}
+
+size_t parallax_decode_workspace_bytes(int B, int Hq, int Hkv, int D, int Lmax, int num_splits) {
+  if (!shape_ok(B, Hq, Hkv, D, Lmax) || (D != 64 && D != 128)) return 0;
+  int P = 0;
+  if (resolve_splits(num_splits, B, Hkv, Lmax, &P) != PARALLAX_OK) return 0;
+  return workspace_bytes_for(Hq / Hkv, D, P);
+}
+
+int parallax_decode(const void* q, const void* r, const void* k_cache, const void* v_cache,
+                    const int32_t* cache_seqlens, void* out, int B, int Hq, int Hkv, int D,
+                    float scale, void* stream, int Lmax, int in_dtype, int out_dtype,
+                    int num_splits, void* workspace, size_t workspace_bytes) {
+  return run(make_call(3, true, q, r, k_cache, v_cache, cache_seqlens, out, B, Hq, Hkv, D, scale,
+                       stream, Lmax, in_dtype, out_dtype, num_splits, workspace, workspace_bytes));
+}
+
+int parallax_softmax_decode(const void* q, const void* k_cache, const void* v_cache,
+                            const int32_t* cache_seqlens, void* out, int B, int Hq, int Hkv, int D,
+                            float scale, void* stream, int Lmax, int in_dtype, int out_dtype,
+                            int num_splits, void* workspace, size_t workspace_bytes) {
+  return run(make_call(3, false, q, nullptr, k_cache, v_cache, cache_seqlens, out, B, Hq, Hkv, D,
+                       scale, stream, Lmax, in_dtype, out_dtype, num_splits, workspace,
+                       workspace_bytes));
+}
+
+int parallax_decode_phase(int phase, int probe, const void* q, const void* r, const void* k_cache,
+                          const void* v_cache, const int32_t* cache_seqlens, void* out, int B,
+                          int Hq, int Hkv, int D, float scale, void* stream, int Lmax, int in_dtype,
+                          int out_dtype, int num_splits, void* workspace, size_t workspace_bytes) {
+  if (phase != 1 && phase != 2) return PARALLAX_ERR_BAD_PHASE;
+  return run(make_call(phase, probe != 0, q, r, k_cache, v_cache, cache_seqlens, out, B, Hq, Hkv,
+                       D, scale, stream, Lmax, in_dtype, out_dtype, num_splits, workspace,
+                       workspace_bytes));
+}
+
+int parallax_workspace_status(void* workspace, int clear, uint32_t* device_status) {
+  if (!workspace || !device_status) return PARALLAX_ERR_NULL_POINTER;
+  uint32_t word = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess) return PARALLAX_ERR_CUDA;
+  if (cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return PARALLAX_ERR_CUDA;
+  if (clear && cudaMemset(workspace, 0, sizeof(word)) != cudaSuccess) return PARALLAX_ERR_CUDA;
+  *device_status = word;
+  if (word & PARALLAX_DEVICE_STATUS_TIMEOUT) return PARALLAX_ERR_DEVICE_TIMEOUT;
+  if (word & PARALLAX_DEVICE_STATUS_SEQLEN_CLAMPED) return PARALLAX_ERR_SEQLEN_CLAMPED;
+  return PARALLAX_OK;
+}
+
+const char* parallax_status_string(int status) {
+  switch (status) {
+    case PARALLAX_OK: return "ok";
+    case PARALLAX_ERR_NULL_POINTER: return "a required pointer is NULL";
+    case PARALLAX_ERR_BAD_SHAPE: return "bad shape (B, Hq, Hkv, Lmax >= 1 and Hq % Hkv == 0 required)";
+    case PARALLAX_ERR_UNSUPPORTED_HEAD_DIM: return "unsupported head dimension (64 or 128)";
+    case PARALLAX_ERR_UNSUPPORTED_DTYPE: return "unsupported dtype selector";
+    case PARALLAX_ERR_MISALIGNED: return "a pointer is not 16-byte aligned";
+    case PARALLAX_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case PARALLAX_ERR_BAD_SPLITS: return "num_splits out of range";
+    case PARALLAX_ERR_CUDA: return "CUDA runtime error (launch or descriptor encoding)";
+    case PARALLAX_ERR_DEVICE_TIMEOUT: return "a bounded wait inside a kernel timed out";
+    case PARALLAX_ERR_BAD_PHASE: return "phase must be 1 or 2";
+    case PARALLAX_ERR_SEQLEN_CLAMPED: return "a cache_seqlens value was outside [0, Lmax] and was clamped";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,113 @@
+"""The C ABI on the host: the library loads, exports every entry point the
+header declares, and rejects bad arguments before touching a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from parameterized_local_linear_b200 import binding, build
+
+HEADER = os.path.join(os.path.dirname(build.PKG), "include", "parallax.h")
+
+OK, ENULL, ESHAPE, EHEAD, EDTYPE, EALIGN, EWS, ESPLITS = 0, -1, -2, -3, -4, -5, -6, -7
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return binding.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(parallax_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("parallax_decode", "parallax_softmax_decode", "parallax_decode_phase",
+                     "parallax_decode_workspace_bytes", "parallax_choose_splits",
+                     "parallax_status_string", "parallax_workspace_status"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} declared in parallax.h but not exported"
+
+
+def test_header_compiles_as_c(tmp_path):
+    src = tmp_path / "t.c"
+    src.write_text('#include "parallax.h"\nint main(void){return PARALLAX_OK;}\n')
+    import subprocess
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.dirname(HEADER),
+                    "-c", str(src), "-o", str(tmp_path / "t.o")], check=True)
+
+
+def test_status_strings(lib):
+    for code in range(-11, 1):
+        s = binding.parallax_status_string(code)
+        assert s and s != "unknown status"
+    assert binding.parallax_status_string(-99) == "unknown status"
+
+
+def test_choose_splits_host_only(lib):
+    # explicit SM count: pure host arithmetic
+    assert lib.parallax_choose_splits(1, 8, 4096, 148) == 296
+    assert lib.parallax_choose_splits(2048, 8, 4096, 148) == 296
+    assert lib.parallax_choose_splits(1, 1, 1, 148) == 1
+    assert lib.parallax_choose_splits(2, 2, 128, 148) == 8  # 512 keys / 64
+    assert lib.parallax_choose_splits(0, 8, 4096, 148) == ESHAPE
+
+
+def test_workspace_bytes_host_only(lib):
+    # 256-byte header + 2 records per split and query head of a group
+    G, D, P = 2, 128, 10
+    want = 256 + 2 * P * G * (4 + 2 * D) * 4
+    assert lib.parallax_decode_workspace_bytes(1, 16, 8, 128, 4096, P) == want
+    assert lib.parallax_decode_workspace_bytes(1, 16, 8, 96, 4096, P) == 0  # D
+    assert lib.parallax_decode_workspace_bytes(1, 15, 8, 128, 4096, P) == 0  # Hq % Hkv
+    assert lib.parallax_decode_workspace_bytes(1, 16, 8, 128, 4096, -1) == 0
+
+
+def _call(lib, **kw):
+    a = dict(q=16, r=16, k=16, v=16, n=16, out=16, B=1, Hq=16, Hkv=8, D=128, scale=0.1,
+             stream=None, Lmax=64, ind=0, outd=0, splits=4, ws=16, wsb=1 << 20)
+    a.update(kw)
+    return lib.parallax_decode(a["q"], a["r"], a["k"], a["v"], a["n"], a["out"], a["B"], a["Hq"],
+                               a["Hkv"], a["D"], ctypes.c_float(a["scale"]), a["stream"],
+                               a["Lmax"], a["ind"], a["outd"], a["splits"], a["ws"], a["wsb"])
+
+
+def test_argument_errors_before_launch(lib):
+    # Fake, aligned, never dereferenced addresses: each call fails validation
+    # on the host, so nothing reaches the device.
+    assert _call(lib, q=None) == ENULL
+    assert _call(lib, r=None) == ENULL
+    assert _call(lib, ws=None) == ENULL
+    assert _call(lib, Hq=12) == ESHAPE
+    assert _call(lib, B=0) == ESHAPE
+    assert _call(lib, Lmax=0) == ESHAPE
+    assert _call(lib, D=96) == EHEAD
+    assert _call(lib, ind=2) == EDTYPE
+    assert _call(lib, outd=-1) == EDTYPE
+    assert _call(lib, k=24) == EALIGN
+    assert _call(lib, out=8) == EALIGN
+    assert _call(lib, n=18) == EALIGN
+    assert _call(lib, splits=-1) == ESPLITS
+    assert _call(lib, splits=65537) == ESPLITS
+    assert _call(lib, wsb=100) == EWS  # explicit splits: sized on the host
+
+
+def test_softmax_decode_does_not_need_r(lib):
+    rc = lib.parallax_softmax_decode(16, 16, 16, 16, 16, 1, 16, 8, 128, ctypes.c_float(0.1),
+                                     None, 64, 0, 0, 4, 16, 100)
+    assert rc == EWS  # got past the pointer checks without r
+
+
+def test_phase_selector(lib):
+    rc = lib.parallax_decode_phase(3, 1, 16, 16, 16, 16, 16, 16, 1, 16, 8, 128,
+                                   ctypes.c_float(0.1), None, 64, 0, 0, 4, 16, 1 << 20)
+    assert rc == -10
