@@ -160,6 +160,46 @@ int parallax_workspace_status(void* workspace, int clear, uint32_t* device_statu
 /* Human-readable text for a status code; never NULL. */
 const char* parallax_status_string(int status);
 
+/*
+ * parallax_decode_noalloc - parallax_decode for callers that cannot allocate.
+ *
+ * The paper has no counterpart to this entry point; it exists for callers of
+ * this library that have no way to obtain device memory for the workspace:
+ * for example a plugin or C host program running next to a framework whose
+ * memory pool has already reserved the GPU's memory, or a latency-critical
+ * decode loop that must never call cudaMalloc (which can synchronise the
+ * device and fail once a pool holds everything). Such callers pass only the
+ * inputs and the output; the workspace is a fixed array of
+ * PARALLAX_NOALLOC_SCRATCH_BYTES in the library's own device memory, which
+ * every GPU that loads the library holds until the process exits.
+ *
+ *  - Arguments are those of parallax_decode without workspace and
+ *    workspace_bytes; the same layouts, dtypes and errors apply.
+ *  - A call whose workspace (parallax_decode_workspace_bytes for the same
+ *    shape and num_splits) would exceed PARALLAX_NOALLOC_SCRATCH_BYTES is
+ *    rejected with PARALLAX_ERR_SCRATCH_LIMIT before anything is launched.
+ *    With D = 128 the array holds 1008 partitions for 2 query heads per kv
+ *    head, 504 for 4 and 252 for 8 (the default is 2 per SM, 296 on a B200);
+ *    pass a smaller num_splits for larger groups.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - Every call on a device shares the one array and leaves its contents
+ *    behind; each call clears the status word at its start (a
+ *    cudaMemsetAsync on `stream`). Calls that can overlap on the GPU (other
+ *    streams, other host threads) race on the array: order them.
+ *  - Device-side status (bounded-wait timeouts, clamped lengths) is kept in
+ *    the array and not reported; use parallax_decode to read it.
+ *  - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ */
+#define PARALLAX_NOALLOC_SCRATCH_BYTES (4u << 20)
+#define PARALLAX_ERR_SCRATCH_LIMIT (-12)
+int parallax_decode_noalloc(const void* q, const void* r, const void* k_cache,
+                            const void* v_cache, const int32_t* cache_seqlens,
+                            void* out, int B, int Hq, int Hkv, int D, float scale,
+                            void* stream, int Lmax, int in_dtype, int out_dtype,
+                            int num_splits);
+
 #ifdef __cplusplus
 }
 #endif

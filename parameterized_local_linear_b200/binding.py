@@ -190,3 +190,27 @@ def parallax_decode_phase(phase: int, probe: bool, q, r, k_cache, v_cache, cache
         _DTYPE_CODE[out.dtype], int(num_splits), workspace.ptr(), workspace.nbytes)
     _check(rc, "parallax_decode_phase")
     return out
+
+
+def parallax_decode_noalloc(q, r, k_cache, v_cache, cache_seqlens, scale: Optional[float] = None,
+                            out=None, out_dtype=None, num_splits: int = 0, stream=None):
+    """parallax_decode without a caller workspace, for callers that cannot
+    allocate device memory: the library uses its own fixed device array (see
+    include/parallax.h). Calls that can overlap on the GPU race on it."""
+    lib = load_library()
+    fn = lib.parallax_decode_noalloc
+    vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    fn.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, f, vp, i, i, i, i]
+    fn.restype = i
+    B, Hq, Hkv, D, Lmax = _shapes(q, k_cache, v_cache, cache_seqlens)
+    if out is None:
+        out = torch.empty((B, Hq, D), device=q.device,
+                          dtype=out_dtype if out_dtype is not None else q.dtype)
+    if r.shape != q.shape or r.dtype != q.dtype or not r.is_cuda or not r.is_contiguous():
+        raise ValueError("r must be a contiguous CUDA tensor shaped like q")
+    scale = D ** -0.5 if scale is None else scale
+    rc = fn(q.data_ptr(), r.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+            cache_seqlens.data_ptr(), out.data_ptr(), B, Hq, Hkv, D, float(scale),
+            _stream(stream), Lmax, _DTYPE_CODE[q.dtype], _DTYPE_CODE[out.dtype], int(num_splits))
+    _check(rc, "parallax_decode_noalloc")
+    return out

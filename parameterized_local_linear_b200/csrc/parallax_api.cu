@@ -356,8 +356,64 @@ const char* parallax_status_string(int status) {
     case PARALLAX_ERR_DEVICE_TIMEOUT: return "a bounded wait inside a kernel timed out";
     case PARALLAX_ERR_BAD_PHASE: return "phase must be 1 or 2";
     case PARALLAX_ERR_SEQLEN_CLAMPED: return "a cache_seqlens value was outside [0, Lmax] and was clamped";
+    case PARALLAX_ERR_SCRATCH_LIMIT:
+      return "the workspace this call needs exceeds PARALLAX_NOALLOC_SCRATCH_BYTES (lower num_splits)";
     default: return "unknown status";
   }
 }
 
 }  // extern "C"
+
+// --------------------------------------------------------------------------
+// parallax_decode_noalloc: the same decode for callers that cannot allocate
+// device memory (see include/parallax.h). Its workspace is this file-scope
+// array in the library's device memory. In host code the array's name is
+// only a host-side stand-in, so the device address is looked up once per
+// device with cudaGetSymbolAddress and passed to the kernels like any
+// caller-provided workspace.
+namespace {
+
+constexpr size_t kNoallocScratchBytes = PARALLAX_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
+
+std::mutex g_noalloc_mutex;
+void* g_noalloc_addr[256] = {};
+
+// Device address of g_noalloc_scratch on the current device (first call per
+// device does the lookup, with that device current).
+int noalloc_scratch_address(void** addr) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 256) return PARALLAX_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return PARALLAX_ERR_CUDA;
+    g_noalloc_addr[dev] = p;
+  }
+  *addr = g_noalloc_addr[dev];
+  return PARALLAX_OK;
+}
+
+}  // namespace
+
+extern "C" int parallax_decode_noalloc(const void* q, const void* r, const void* k_cache,
+                                       const void* v_cache, const int32_t* cache_seqlens,
+                                       void* out, int B, int Hq, int Hkv, int D, float scale,
+                                       void* stream, int Lmax, int in_dtype, int out_dtype,
+                                       int num_splits) {
+  void* scratch = nullptr;
+  int st = noalloc_scratch_address(&scratch);
+  if (st != PARALLAX_OK) return st;
+  Call c = make_call(3, true, q, r, k_cache, v_cache, cache_seqlens, out, B, Hq, Hkv, D, scale,
+                     stream, Lmax, in_dtype, out_dtype, num_splits, scratch, kNoallocScratchBytes);
+  if ((st = validate(c)) != PARALLAX_OK) return st;
+  int P = 0;
+  if ((st = resolve_splits(num_splits, B, Hkv, Lmax, &P)) != PARALLAX_OK) return st;
+  if (workspace_bytes_for(Hq / Hkv, D, P) > kNoallocScratchBytes) return PARALLAX_ERR_SCRATCH_LIMIT;
+  // The array keeps the previous call's contents: the status word must start
+  // at zero; the partial records are always written before they are read.
+  if (cudaMemsetAsync(scratch, 0, kWorkspaceHeaderBytes, c.stream) != cudaSuccess)
+    return PARALLAX_ERR_CUDA;
+  return run(c);
+}
