@@ -35,36 +35,50 @@ constexpr int kConsumerWarps = 4;    // each owns 16 keys of a stage
 constexpr int kTcThreads = (kConsumerWarps + 1) * 32;  // + one producer warp
 constexpr int kBoxBytes = kTileKeys * 128;             // one 64-key x 128-byte swizzled box
 
+// A 96 KB ring of K+V per CTA: measured on B200, one CTA per SM with 96 KB
+// in flight streams faster than 192 KB per SM (one CTA with a 6-stage ring,
+// or two CTAs), and it leaves shared memory for the merge kernel's blocks to
+// become resident early.
 template <int D>
 struct TcGeom {
   static constexpr int kHalves = D / 64;                 // 128-byte boxes per key row
   static constexpr int kKBytes = kHalves * kBoxBytes;    // K tile of one stage
   static constexpr int kStageBytes = 2 * kKBytes;        // K + V
-  static constexpr int kStages = D == 128 ? 3 : 6;       // 96 KB of ring either way
+  static constexpr int kStages = D == 128 ? 3 : 6;
 };
 
 __host__ __device__ constexpr int align_up(int x, int a) { return (x + a - 1) / a * a; }
 
 // Byte offsets inside the (1024-aligned) dynamic shared memory of the TMA kernel.
 struct TcSmemLayout {
-  int qr_slot_bytes, off_qr, off_p, off_merge, off_bar, off_misc, total;
+  int off_p, off_merge, off_bar, off_misc, total;
 };
 
 __host__ __device__ inline TcSmemLayout tc_smem_layout(int D, int stage_bytes, int stages, int G,
                                                        bool probe) {
+  (void)probe;
   TcSmemLayout L{};
-  L.qr_slot_bytes = align_up((probe ? 2 : 1) * G * D * 2, 128);
-  L.off_qr = stages * stage_bytes;
-  L.off_p = L.off_qr + 2 * L.qr_slot_bytes;
+  L.off_p = stages * stage_bytes;
   L.off_merge = L.off_p + kConsumerWarps * 512;
   L.off_bar = align_up(L.off_merge + kConsumerWarps * G * rec_floats(D) * 4, 16);
-  // full[stages], empty[stages], qr_full[2], qr_empty[2], fin[2]
-  L.off_misc = L.off_bar + 8 * (2 * stages + 6);
-  L.total = L.off_misc + 512 + 1024;  // prologue scratch, abort flag, alignment slack
+  // full[stages], empty[stages], fin[2]
+  L.off_misc = L.off_bar + 8 * (2 * stages + 2);
+  L.total = L.off_misc + 16 + 1024;  // abort flag, alignment slack
   return L;
 }
 
 constexpr int kGenericThreads = 128;
-constexpr int kMergeThreads = 128;
+constexpr int kMergeThreads = 256;
+constexpr int kMergeMaxG = 128;        // query heads per kv head handled by the merge kernel
+constexpr int kMergeColsPerBlock = 32; // float4 columns of A/C one merge block sums
+constexpr int kMergeMaxPerThread = 4;  // records one thread loads in the one-pass merge
+
+// Merge blocks per partition: the owner's (head, 4-dim) output groups times
+// (A, C) are split so that each block sums about kMergeColsPerBlock float4
+// columns (never more than kMergeThreads).
+__host__ __device__ inline int merge_slices(int G, int D, bool probe) {
+  const int cols = G * (D / 4) * (probe ? 2 : 1);
+  return (cols + kMergeColsPerBlock - 1) / kMergeColsPerBlock;
+}
 
 }  // namespace plx

@@ -34,13 +34,13 @@ __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) {
 template <typename T, bool PROBE, bool OUT_F32>
 __global__ void __launch_bounds__(kGenericThreads)
     parallax_generic_kernel(const DecodeParams p) {
-  __shared__ PrologueScratch scratch;
   __shared__ float s_t[kGenericThreads];
   __shared__ float s_s[kGenericThreads];
   const float kNegInf = __int_as_float(0xff800000u);
 
-  const PartitionInfo part = locate_partition<kGenericThreads>(p.seqlens, p.B, p.Hkv, p.Lmax,
-                                                               blockIdx.x, gridDim.x, &scratch);
+  pdl_wait_primary();  // launched with programmatic stream serialisation
+  const PartitionInfo part =
+      locate_partition(p.seqlens, p.B, p.Hkv, p.Lmax, blockIdx.x, gridDim.x);
   if (blockIdx.x == 0 && threadIdx.x == 0 && part.clamped) atomicOr(p.status, 2u);
   pdl_launch_dependents();
   if (part.lo >= part.hi) return;

@@ -2,12 +2,14 @@
 //
 // One CTA per partition of the flattened key range (see partition.cuh),
 // persistent over the pieces of that range. Warp 4 is the producer: one lane
-// streams 64-key K and V tiles of the current item with TMA (3-D tensor maps
-// over [B*Hkv][Lmax][D], 128-byte swizzle, no multicast) into a ring of
-// shared-memory stages guarded by full/empty mbarriers, and bulk-copies the
-// q (and r) rows of the item's GQA group. Warps 0..3 consume: warp w owns
-// keys 16w..16w+15 of every stage and keeps its own online accumulators, so
-// the consumer warps never synchronise inside the key loop.
+// streams 64-key K and V tiles of the current item with one TMA each (4-D
+// tensor maps over the [B*Hkv][Lmax][D] caches, 128-byte swizzle, no
+// multicast) into a ring of shared-memory stages guarded by full/empty
+// mbarriers. Warps 0..3 consume: warp w owns keys 16w..16w+15 of every stage
+// and keeps its own online accumulators, so the consumer warps never
+// synchronise inside the key loop. They read the q (and r) rows of the item's
+// GQA group straight into mma fragments from global memory, overlapped with
+// the first K/V tile's flight.
 //
 // The method streams the same K/V tiles as FlashAttention and does twice its
 // work per byte ("Parallax: Parameterized Local Linear Attention for Language
@@ -41,7 +43,7 @@
 namespace plx {
 
 template <int D, bool PROBE, bool OUT_F32, bool PSPLIT>
-__global__ void __launch_bounds__(kTcThreads, 2)
+__global__ void __launch_bounds__(kTcThreads, 1)
     parallax_tc_kernel(const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const DecodeParams p) {
   static_assert(!PROBE || PSPLIT, "the probe kernel needs the hi + lo split of P");
@@ -60,11 +62,8 @@ __global__ void __launch_bounds__(kTcThreads, 2)
 
   const uint32_t bar_full = base + L.off_bar;
   const uint32_t bar_empty = bar_full + 8 * kStages;
-  const uint32_t bar_qr_full = bar_empty + 8 * kStages;
-  const uint32_t bar_qr_empty = bar_qr_full + 16;
-  const uint32_t bar_fin = bar_qr_empty + 16;
-  PrologueScratch* scratch = reinterpret_cast<PrologueScratch*>(gbase + L.off_misc);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L.off_misc + sizeof(PrologueScratch));
+  const uint32_t bar_fin = bar_empty + 8 * kStages;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L.off_misc);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
@@ -72,56 +71,41 @@ __global__ void __launch_bounds__(kTcThreads, 2)
       mbar_init(bar_full + 8 * s, 1);
       mbar_init(bar_empty + 8 * s, kConsumerWarps);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(bar_qr_full + 8 * s, 1);
-      mbar_init(bar_qr_empty + 8 * s, kConsumerWarps);
-      mbar_init(bar_fin + 8 * s, kConsumerWarps * 32);
-    }
+    for (int s = 0; s < 2; ++s) mbar_init(bar_fin + 8 * s, kConsumerWarps);
     *abort_flag = 0;
     mbar_fence_init();
   }
+  uint64_t policy = 0;
+  if (tid == kConsumerWarps * 32) {  // the producer lane: descriptors are kernel parameters
+    prefetch_tensormap(&tmK);
+    prefetch_tensormap(&tmV);
+    policy = l2_policy_evict_first();
+  }
+  __syncthreads();  // barriers initialised before anyone uses them
+  // Launched with programmatic stream serialisation: everything above overlaps
+  // the previous kernel in the stream; nothing below may run before it ends.
+  pdl_wait_primary();
   const PartitionInfo part =
-      locate_partition<kTcThreads>(p.seqlens, p.B, p.Hkv, p.Lmax, blockIdx.x, gridDim.x, scratch);
+      locate_partition(p.seqlens, p.B, p.Hkv, p.Lmax, blockIdx.x, gridDim.x);
   if (blockIdx.x == 0 && tid == 0 && part.clamped)
     atomicOr(p.status, 2u /* PARALLAX_DEVICE_STATUS_SEQLEN_CLAMPED */);
-  pdl_launch_dependents();
+  // The merge grid may be scheduled once every CTA has its first stage in
+  // flight (threads that return early count as triggered): early enough to
+  // hide its prologue, late enough not to slow this kernel's start.
   if (part.lo >= part.hi) return;
 
   const int G = p.G;
-  const uint32_t qr_row_bytes = (uint32_t)G * D * 2;
 
   // ------------------------------------------------------------ producer --
   if (warp == kConsumerWarps) {
     if (lane != 0) return;
-    prefetch_tensormap(&tmK);
-    prefetch_tensormap(&tmV);
-    const uint64_t policy = l2_policy_evict_first();
     PieceCursor cur;
     cur.init(part, p.seqlens, p.B, p.Hkv, p.Lmax);
     Piece pc;
-    int stage = 0, qs = 0;
-    uint32_t ph = 0, qph = 0;
-    uint32_t issued_mask = 0, issued_par = 0, qr_issued_mask = 0, qr_issued_par = 0;
+    int stage = 0;
+    uint32_t ph = 0, issued_mask = 0, issued_par = 0;
     bool ok = true, skip = p.debug_skip_first_tile != 0;
     while (ok && cur.next(pc)) {
-      if (!mbar_wait_bounded(bar_qr_empty + 8 * qs, qph ^ 1, p.timeout_ns, abort_flag)) {
-        ok = false;
-        break;
-      }
-      const size_t row0 = ((size_t)pc.b * p.Hq + (size_t)pc.g * G) * D;
-      mbar_arrive_expect_tx(bar_qr_full + 8 * qs, (PROBE ? 2 : 1) * qr_row_bytes);
-      const uint32_t qr_dst = base + L.off_qr + qs * L.qr_slot_bytes;
-      bulk_load(qr_dst, static_cast<const __nv_bfloat16*>(p.q) + row0, qr_row_bytes,
-                bar_qr_full + 8 * qs);
-      if (PROBE)
-        bulk_load(qr_dst + qr_row_bytes, static_cast<const __nv_bfloat16*>(p.r) + row0,
-                  qr_row_bytes, bar_qr_full + 8 * qs);
-      qr_issued_mask |= 1u << qs;
-      qr_issued_par = (qr_issued_par & ~(1u << qs)) | (qph << qs);
-      if (++qs == 2) {
-        qs = 0;
-        qph ^= 1;
-      }
       const int item = pc.b * p.Hkv + pc.g;
       for (int k0 = pc.i; k0 < pc.i + pc.len; k0 += kTileKeys) {
         if (!mbar_wait_bounded(bar_empty + 8 * stage, ph ^ 1, p.timeout_ns, abort_flag)) {
@@ -134,12 +118,9 @@ __global__ void __launch_bounds__(kTcThreads, 2)
           const uint32_t full = bar_full + 8 * stage;
           const uint32_t sK = base + stage * kStageBytes;
           mbar_arrive_expect_tx(full, kStageBytes);
-#pragma unroll
-          for (int h = 0; h < Geom::kHalves; ++h)
-            tma_load_3d(sK + h * kBoxBytes, &tmK, 64 * h, k0, item, full, policy);
-#pragma unroll
-          for (int h = 0; h < Geom::kHalves; ++h)
-            tma_load_3d(sK + kKBytes + h * kBoxBytes, &tmV, 64 * h, k0, item, full, policy);
+          tma_load_4d(sK, &tmK, 0, k0, 0, item, full, policy);
+          tma_load_4d(sK + kKBytes, &tmV, 0, k0, 0, item, full, policy);
+          if (issued_mask == 0) pdl_launch_dependents();
           issued_mask |= 1u << stage;
           issued_par = (issued_par & ~(1u << stage)) | (ph << stage);
         }
@@ -149,6 +130,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         }
       }
     }
+    if (issued_mask == 0) pdl_launch_dependents();
     if (!ok) {
       // Give up: tell the consumers, record the timeout, and wait (bounded)
       // for this CTA's copies still in flight before leaving.
@@ -157,9 +139,6 @@ __global__ void __launch_bounds__(kTcThreads, 2)
       for (int s = 0; s < kStages; ++s)
         if (issued_mask & (1u << s))
           mbar_wait_bounded(bar_full + 8 * s, (issued_par >> s) & 1u, p.timeout_ns, nullptr);
-      for (int s = 0; s < 2; ++s)
-        if (qr_issued_mask & (1u << s))
-          mbar_wait_bounded(bar_qr_full + 8 * s, (qr_issued_par >> s) & 1u, p.timeout_ns, nullptr);
     }
     return;
   }
@@ -183,42 +162,31 @@ __global__ void __launch_bounds__(kTcThreads, 2)
   PieceCursor cur;
   cur.init(part, p.seqlens, p.B, p.Hkv, p.Lmax);
   Piece pc;
-  int stage = 0, qs = 0;
-  uint32_t ph = 0, qph = 0, fph = 0;
-  bool ok = true;
+  int stage = 0;
+  uint32_t ph = 0, fph = 0;
+  bool ok = true, triggered = false;
 
   while (ok && cur.next(pc)) {
     // --- B fragments of the group's q (and r) rows; column n = lane / 4 ---
-    if (!mbar_wait_bounded(bar_qr_full + 8 * qs, qph, p.timeout_ns, abort_flag)) {
-      ok = false;
-      break;
-    }
     uint32_t bq[kJ][2];
     {
-      const uint8_t* qr = gbase + L.off_qr + qs * L.qr_slot_bytes;
-      int h, off;
+      int h, is_r;
       if (PROBE) {
         h = g8 >> 1;
-        off = (g8 & 1) * G * D;  // odd columns read the probe rows
+        is_r = g8 & 1;  // odd columns hold the probe rows
       } else {
         h = g8;
-        off = 0;
+        is_r = 0;
       }
-      const bool valid = h < G;
-      const uint16_t* row = reinterpret_cast<const uint16_t*>(qr) + off + (valid ? h : 0) * D;
+      const bool valid = h < G;  // columns past the group stay zero
+      const size_t row = ((size_t)pc.b * p.Hq + (size_t)pc.g * G + (valid ? h : 0)) * D;
+      const uint32_t* src = reinterpret_cast<const uint32_t*>(
+          static_cast<const __nv_bfloat16*>(is_r ? p.r : p.q) + row);
 #pragma unroll
       for (int j = 0; j < kJ; ++j) {
-        const uint32_t b0 = *reinterpret_cast<const uint32_t*>(row + 16 * j + 2 * c4);
-        const uint32_t b1 = *reinterpret_cast<const uint32_t*>(row + 16 * j + 2 * c4 + 8);
-        bq[j][0] = valid ? b0 : 0u;
-        bq[j][1] = valid ? b1 : 0u;
+        bq[j][0] = valid ? __ldg(src + 8 * j + c4) : 0u;      // dims 16j + 2c4, +1
+        bq[j][1] = valid ? __ldg(src + 8 * j + c4 + 4) : 0u;  // dims 16j + 2c4 + 8, +9
       }
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(bar_qr_empty + 8 * qs);
-    if (++qs == 2) {
-      qs = 0;
-      qph ^= 1;
     }
 
     float acc[kJ][4];
@@ -233,6 +201,10 @@ __global__ void __launch_bounds__(kTcThreads, 2)
       if (!mbar_wait_bounded(bar_full + 8 * stage, ph, p.timeout_ns, abort_flag)) {
         ok = false;
         break;
+      }
+      if (!triggered) {
+        pdl_launch_dependents();
+        triggered = true;
       }
       const int nvalid = min(kTileKeys, pc.i + pc.len - k0);
       const uint32_t sK = base + stage * kStageBytes;
@@ -440,7 +412,8 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         }
       }
     }
-    mbar_arrive(bar_fin);  // every consumer thread: publishes its scratch writes
+    __syncwarp();  // orders the warp's scratch writes before lane 0's release
+    if (lane == 0) mbar_arrive(bar_fin);
     if (!mbar_wait_bounded(bar_fin, fph, p.timeout_ns, abort_flag)) {
       ok = false;
       break;
@@ -486,13 +459,15 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         }
       }
     }
-    mbar_arrive(bar_fin + 8);  // scratch may be overwritten by the next piece
+    __syncwarp();  // scratch may be overwritten by the next piece
+    if (lane == 0) mbar_arrive(bar_fin + 8);
     if (!mbar_wait_bounded(bar_fin + 8, fph, p.timeout_ns, abort_flag)) {
       ok = false;
       break;
     }
     fph ^= 1;
   }
+  if (!triggered) pdl_launch_dependents();
   if (!ok) {
     *abort_flag = 1;
     if (lane == 0) atomicOr(p.status, 1u /* PARALLAX_DEVICE_STATUS_TIMEOUT */);

@@ -22,8 +22,8 @@ using namespace plx;
 namespace {
 
 constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;  // 2 s per wait
-constexpr long long kMinKeysPerSplit = 64;  // smallest key range worth a CTA
-constexpr int kCtasPerSm = 2;               // split-KV CTAs resident per SM
+constexpr long long kMinKeysPerSplit = 256;  // smallest key range worth a CTA
+constexpr int kCtasPerSm = 1;                // split-KV CTAs per SM (96 KB ring each)
 
 struct Call {
   int phases;  // bit 0: split-KV kernel, bit 1: merge kernel
@@ -69,7 +69,9 @@ int choose_splits_impl(int B, int Hkv, int Lmax, int sm_count) {
 bool shape_ok(int B, int Hq, int Hkv, int D, int Lmax) {
   if (B < 1 || Hq < 1 || Hkv < 1 || Lmax < 1 || D < 1) return false;
   if (Hq % Hkv != 0) return false;
-  if ((long long)B * Hkv > 0x7fffffffLL) return false;  // TMA item coordinate is int32
+  if (Hq / Hkv > kMergeMaxG) return false;  // query heads per kv head
+  if ((long long)B * Hkv > 0x7fffffffLL) return false;     // TMA item coordinate is int32
+  if ((long long)Hkv * Lmax > 0x7fffffffLL) return false;  // key offsets inside a batch row
   return true;
 }
 
@@ -121,15 +123,17 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// [B*Hkv][Lmax][D] bf16 cache, boxes of 64 keys x 64 dims (128 bytes, swizzled).
+// [B*Hkv][Lmax][D] bf16 cache viewed as {64 dims, Lmax keys, D/64 halves,
+// B*Hkv items}: one box of 64 keys x D dims lands as D/64 swizzled
+// [64 keys][128 bytes] blocks, one per 64-dim half.
 int encode_cache_map(CUtensorMap* map, const void* cache, int D, int Lmax, long long items) {
   auto enc = tensor_map_encoder();
   if (!enc) return PARALLAX_ERR_CUDA;
-  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Lmax, (cuuint64_t)items};
-  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)Lmax * D * 2};
-  cuuint32_t box[3] = {64, (cuuint32_t)kTileKeys, 1};
-  cuuint32_t elem[3] = {1, 1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(cache), dims,
+  cuuint64_t dims[4] = {64, (cuuint64_t)Lmax, (cuuint64_t)(D / 64), (cuuint64_t)items};
+  cuuint64_t strides[3] = {(cuuint64_t)D * 2, 128, (cuuint64_t)Lmax * D * 2};
+  cuuint32_t box[4] = {64, (cuuint32_t)kTileKeys, (cuuint32_t)(D / 64), 1};
+  cuuint32_t elem[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(cache), dims,
                    strides, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? PARALLAX_OK : PARALLAX_ERR_CUDA;
@@ -163,21 +167,31 @@ int launch_tc(const Call& c, const DecodeParams& prm, int P) {
   const long long items = (long long)c.B * c.Hkv;
   if ((st = encode_cache_map(&tmK, c.k, D, c.Lmax, items)) != PARALLAX_OK) return st;
   if ((st = encode_cache_map(&tmV, c.v, D, c.Lmax, items)) != PARALLAX_OK) return st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)P);
   cfg.blockDim = dim3(kTcThreads);
   cfg.dynamicSmemBytes = (size_t)L.total;
   cfg.stream = c.stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kernel, tmK, tmV, prm) == cudaSuccess ? PARALLAX_OK
                                                                         : PARALLAX_ERR_CUDA;
 }
 
 template <typename T, bool PROBE, bool OUT_F32>
 int launch_generic(const Call& c, const DecodeParams& prm, int P) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)P);
   cfg.blockDim = dim3(kGenericThreads);
   cfg.stream = c.stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, parallax_generic_kernel<T, PROBE, OUT_F32>, prm) == cudaSuccess
              ? PARALLAX_OK
              : PARALLAX_ERR_CUDA;
@@ -189,7 +203,7 @@ int launch_merge(const Call& c, const DecodeParams& prm, int P) {
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)P);
+  cfg.gridDim = dim3((unsigned)P, (unsigned)merge_slices(prm.G, prm.D, PROBE));
   cfg.blockDim = dim3(kMergeThreads);
   cfg.stream = c.stream;
   cfg.attrs = attr;

@@ -26,91 +26,66 @@ struct PartitionInfo {
   long long per;    // keys per partition
   long long lo, hi; // this partition's range
   int b, g, i;      // item and key offset at position lo (valid if lo < hi)
+  int n;            // clamped length of batch b
   int clamped;      // some cache_seqlens value was outside [0, Lmax]
 };
 
-struct PrologueScratch {
-  long long warp_sum[32];
-  long long total;
-  long long within;
-  int b;
-  int clamped;
-};
-
-// Block-cooperative (every thread of the block must call it, NT threads).
-// Reads cache_seqlens once, computes the partition of this block (index c of
-// P) and locates its first key.
-template <int NT>
-__device__ PartitionInfo locate_partition(const int32_t* __restrict__ seqlens, int B, int Hkv,
-                                          int Lmax, int c, int P, PrologueScratch* s) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  constexpr int kWarps = NT / 32;
-  const int chunk = (B + NT - 1) / NT;
-  const int b0 = min(B, tid * chunk), b1 = min(B, b0 + chunk);
+// Warp-cooperative: every warp of a block calls it and gets the same result,
+// with no block barrier and no shared memory. Each lane sums a contiguous
+// chunk of cache_seqlens (read-only path, so the re-reads hit L1), a warp scan
+// gives the prefix sums, and the lane whose chunk holds position lo walks it
+// to find the item there. c is this block's index among P partitions.
+__device__ inline PartitionInfo locate_partition(const int32_t* __restrict__ seqlens, int B,
+                                                 int Hkv, int Lmax, int c, int P) {
+  const int lane = threadIdx.x & 31;
+  const int chunk = (B + 31) / 32;
+  const int b0 = min(B, lane * chunk), b1 = min(B, b0 + chunk);
   long long local = 0;
   int clamped = 0;
   for (int b = b0; b < b1; ++b) {
-    int n = seqlens[b];
+    const int n = __ldg(seqlens + b);
     clamped |= (n < 0 || n > Lmax);
     local += clamp_len(n, Lmax);
   }
-  // inclusive warp scan of `local`
-  long long incl = local;
+  long long incl = local;  // inclusive scan over lanes
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    long long x = __shfl_up_sync(0xffffffffu, incl, o);
+    const long long x = __shfl_up_sync(0xffffffffu, incl, o);
     if (lane >= o) incl += x;
   }
-  clamped = __any_sync(0xffffffffu, clamped);
-  if (tid == 0) {
-    s->b = -1;
-    s->clamped = 0;
-  }
-  if (lane == 31) s->warp_sum[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    long long w = lane < kWarps ? s->warp_sum[lane] : 0;
-    long long wi = w;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      long long x = __shfl_up_sync(0xffffffffu, wi, o);
-      if (lane >= o) wi += x;
-    }
-    if (lane < kWarps) s->warp_sum[lane] = wi - w;  // exclusive warp offsets
-    if (lane == kWarps - 1) s->total = wi;
-  }
-  if (clamped && lane == 0) atomicOr(&s->clamped, 1);
-  __syncthreads();
-  const long long excl = s->warp_sum[warp] + incl - local;  // lengths before b0
   PartitionInfo p;
-  p.total = (long long)Hkv * s->total;
+  p.clamped = __any_sync(0xffffffffu, clamped);
+  p.total = (long long)Hkv * __shfl_sync(0xffffffffu, incl, 31);
   p.per = (p.total + P - 1) / P;
   p.lo = min(p.total, (long long)c * p.per);
   p.hi = min(p.total, p.lo + p.per);
-  // the thread whose batches contain position lo records the item there
-  if (p.lo < p.hi && local > 0) {
-    long long pos = (long long)Hkv * excl;
-    if (p.lo >= pos && p.lo < pos + (long long)Hkv * local) {
-      for (int b = b0; b < b1; ++b) {
-        const long long blk = (long long)Hkv * clamp_len(seqlens[b], Lmax);
-        if (p.lo < pos + blk) {
-          s->b = b;
-          s->within = p.lo - pos;
-          break;
-        }
-        pos += blk;
+  p.b = -1;
+  p.g = p.i = p.n = 0;
+  // the lane whose batches contain position lo finds the item there
+  long long pos = (long long)Hkv * (incl - local);
+  int fb = -1, fn = 0;
+  long long within = 0;
+  if (p.lo < p.hi && p.lo >= pos && p.lo < pos + (long long)Hkv * local) {
+    for (int b = b0; b < b1; ++b) {
+      const int n = clamp_len(__ldg(seqlens + b), Lmax);
+      const long long blk = (long long)Hkv * n;
+      if (p.lo < pos + blk) {
+        fb = b;
+        fn = n;
+        within = p.lo - pos;
+        break;
       }
+      pos += blk;
     }
   }
-  __syncthreads();
-  p.clamped = s->clamped;
-  p.b = s->b;
-  p.g = 0;
-  p.i = 0;
-  if (p.b >= 0) {
-    const int n = clamp_len(seqlens[p.b], Lmax);
-    p.g = (int)(s->within / n);
-    p.i = (int)(s->within % n);
+  const unsigned owner = __ballot_sync(0xffffffffu, fb >= 0);
+  if (owner) {
+    const int src = __ffs(owner) - 1;
+    p.b = __shfl_sync(0xffffffffu, fb, src);
+    p.n = __shfl_sync(0xffffffffu, fn, src);
+    const int w = (int)__shfl_sync(0xffffffffu, within, src);  // < Hkv * n <= Hkv * Lmax
+    p.g = w / p.n;
+    p.i = w - p.g * p.n;
   }
   return p;
 }
@@ -125,7 +100,7 @@ struct Piece {
 
 // Walks the pieces of one partition; every role of a CTA walks the same list.
 struct PieceCursor {
-  int b, g, i;
+  int b, g, i, n;  // n: clamped length of batch b
   long long pos, lo, hi;
   const int32_t* seqlens;
   int B, Hkv, Lmax;
@@ -134,6 +109,7 @@ struct PieceCursor {
     b = p.b;
     g = p.g;
     i = p.i;
+    n = p.n;
     pos = p.lo;
     lo = p.lo;
     hi = p.hi;
@@ -145,7 +121,6 @@ struct PieceCursor {
 
   __device__ bool next(Piece& pc) {
     if (pos >= hi) return false;
-    const int n = clamp_len(seqlens[b], Lmax);
     const long long room = hi - pos;
     const int len = (long long)(n - i) < room ? n - i : (int)room;
     pc.b = b;
@@ -162,7 +137,8 @@ struct PieceCursor {
       if (++g == Hkv) {
         g = 0;
         ++b;
-        while (pos < hi && b < B && clamp_len(seqlens[b], Lmax) == 0) ++b;
+        n = 0;
+        while (pos < hi && b < B && (n = clamp_len(__ldg(seqlens + b), Lmax)) == 0) ++b;
       }
     }
     return true;
