@@ -34,7 +34,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from parameterized_local_linear_b200 import inputs  # noqa: E402
+from parameterized_local_linear_b200 import inputs, replicas  # noqa: E402
 
 METRIC = "decode µs/step and KV-read GB/s (% of HBM peak) vs in-run R=0 softmax decode"
 FALLBACK_HBM_GBS = 6650.0
@@ -51,6 +51,8 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(inputs.WORKLOADS), default="qwen")
     ap.add_argument("--num-splits", type=int, default=0)
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch size (for profiling a smaller copy)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="bound of the CPU oracle baseline sample (seconds)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -190,15 +192,10 @@ class Dist:
             self.pg = dist
 
     def barrier(self):
-        if self.pg:
-            self.pg.barrier()
+        replicas.barrier()
 
     def max(self, x: float) -> float:
-        if not self.pg:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
-        return float(t.item())
+        return replicas.max_over_ranks(x)
 
     def close(self):
         if self.pg:
@@ -207,37 +204,44 @@ class Dist:
 
 # ------------------------------------------------------------ CPU oracle ----
 
-def oracle_sample(w: inputs.Workload, x_host: dict, budget_s: float):
-    """Time the fp64 oracle, as it stands, on a bounded sample of the workload.
-    Returns (GB/s of KV processed, cores, description, seconds)."""
+def oracle_rows_for_budget(w: inputs.Workload, x_host: dict, budget_s: float):
+    """Batch rows whose single oracle pass takes about budget_s (at least one)."""
     import oracle
-    rows_all = list(range(w.B))
-    lens = x_host["seqlens"].tolist()
-    per_row = [2 * n * w.Hkv * w.D * x_host["k"].element_size() for n in lens]
-    # grow the sample one batch row at a time until its first pass is ~1/5 of the budget
-    done_bytes, elapsed, rows, reps = 0, 0.0, [], 0
-    t_start = time.perf_counter()
-    order = rows_all
-    i = 0
-    while elapsed < budget_s:
-        if i < len(order) and (not rows or elapsed < budget_s / 5):
-            rows.append(order[i])
-            i += 1
-            sel = rows[-1:]
-        else:
-            sel = rows
-            reps += 1
-        idx = torch.tensor(sel)
-        t0 = time.perf_counter()
-        oracle.parallax_decode(x_host["q"][idx], x_host["r"][idx], x_host["k"][idx],
-                               x_host["v"][idx], x_host["seqlens"][idx], x_host["scale"])
-        elapsed += time.perf_counter() - t0
-        done_bytes += sum(per_row[b] for b in sel)
-        if time.perf_counter() - t_start > 3 * budget_s:
-            break
-    desc = (f"fp64 oracle (covariance form) on batch rows {rows[0]}..{rows[-1]} "
-            f"({len(rows)} of {w.B} rows, {reps} extra passes); {elapsed:.1f} s")
-    return done_bytes / elapsed / 1e9, oracle.num_threads(), desc, elapsed
+    idx = torch.tensor([0])
+    t0 = time.perf_counter()
+    oracle.parallax_decode(x_host["q"][idx], x_host["r"][idx], x_host["k"][idx],
+                           x_host["v"][idx], x_host["seqlens"][idx], x_host["scale"])
+    one = max(1e-4, time.perf_counter() - t0)
+    return list(range(max(1, min(w.B, int(budget_s / one)))))
+
+
+def oracle_timed(w: inputs.Workload, x_host: dict, rows, steps: int):
+    """Time `steps` passes of the fp64 oracle, as it stands, over batch rows
+    `rows`. Returns (GB/s of K/V processed, threads, seconds)."""
+    import oracle
+    idx = torch.tensor(rows)
+    sub = {k: (x_host[k][idx] if torch.is_tensor(x_host[k]) else x_host[k])
+           for k in ("q", "r", "k", "v", "seqlens")}
+    n = sub["seqlens"].to(torch.int64).clamp(0, w.Lmax).sum().item()
+    kv = 2 * n * w.Hkv * w.D * x_host["k"].element_size()
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        oracle.parallax_decode(sub["q"], sub["r"], sub["k"], sub["v"], sub["seqlens"],
+                               x_host["scale"])
+    secs = time.perf_counter() - t0
+    return kv * steps / secs / 1e9, oracle.num_threads(), secs
+
+
+def oracle_sample(w: inputs.Workload, x_host: dict, budget_s: float):
+    """The CPU baseline: the oracle on a bounded sample of the workload, about
+    budget_s of CPU work. Returns (GB/s, threads, description, seconds)."""
+    rows = oracle_rows_for_budget(w, x_host, budget_s / 4)
+    _, _, t1 = oracle_timed(w, x_host, rows, 1)
+    passes = max(1, int(budget_s / max(t1, 1e-6)))
+    v, cores, secs = oracle_timed(w, x_host, rows, passes)
+    desc = (f"fp64 oracle (covariance form), {passes} passes over batch rows 0..{rows[-1]} "
+            f"({len(rows)} of {w.B}); {secs:.1f} s")
+    return v, cores, desc, secs
 
 
 def host_inputs_for_oracle(w: inputs.Workload, budget_rows: int = 64):
@@ -256,20 +260,21 @@ def host_inputs_for_oracle(w: inputs.Workload, budget_rows: int = 64):
 
 
 def run_reference(args):
+    """The reference arm: the fp64 CPU oracle on the host cores. A step is one
+    oracle pass over a bounded sample of the workload's batch rows (sized so
+    that the whole run takes a few minutes); exactly K steps are timed."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
     w = inputs.WORKLOADS[args.workload]
     wsub, xh = host_inputs_for_oracle(w)
-    per_step_budget = max(1.0, 120.0 / max(1, args.steps + args.warmup))
-    for _ in range(args.warmup):
-        oracle_sample(wsub, xh, min(per_step_budget, 2.0))
-    vals, secs, desc, cores = [], 0.0, "", 0
-    for _ in range(args.steps):
-        v, cores, desc, s = oracle_sample(wsub, xh, per_step_budget)
-        vals.append(v)
-        secs += s
-    value = statistics.median(vals)
+    per_step = min(5.0, 120.0 / max(1, args.steps + args.warmup))
+    rows = oracle_rows_for_budget(wsub, xh, per_step)
+    if args.warmup:
+        oracle_timed(wsub, xh, rows, args.warmup)
+    value, cores, secs = oracle_timed(wsub, xh, rows, args.steps)
+    desc = (f"fp64 oracle (covariance form); a step = one pass over batch rows 0..{rows[-1]} "
+            f"({len(rows)} of {w.B}) of the workload")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": secs / max(1, args.steps) * 1e3, "higher_is_better": True,
@@ -297,6 +302,9 @@ def main():
     dev = torch.device("cuda", torch.cuda.current_device())
     binding.load_library()
     w = inputs.WORKLOADS[args.workload]
+    if args.batch is not None:
+        w = inputs.Workload(w.name + f"-B{args.batch}", args.batch, w.Hq, w.Hkv, w.D, w.Lmax,
+                            w.dtype, w.seed, w.lengths, w.r_scale, w.k_offset_std, w.scale)
     stream = torch.cuda.Stream(device=dev)  # graphs can not be captured on the legacy stream
     torch.cuda.set_stream(stream)
 
@@ -374,29 +382,66 @@ def main():
     run_soft = make_runner(False)
     sampler = ClockSampler(dev.index)
     t_plx = timed(run_plx, args.steps, args.warmup, sampler)
-    t_soft = timed(run_soft, args.steps, args.warmup)
+
+    # The R = 0 comparator: blocks of Parallax and softmax steps alternate, so
+    # both see the same power and clock state (B200 runs at its power cap
+    # while streaming HBM); the ratio is taken from the block medians.
+    blk = nbuf * max(1, 800 // nbuf) if use_graphs else 10
+    rounds = 8 if use_graphs else 5
+    run_soft(min(args.warmup, blk))
+    per = {True: [], False: []}
+    for _ in range(rounds):
+        for probe, runner in ((True, run_plx), (False, run_soft)):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            runner(blk)
+            b.record(stream)
+            b.synchronize()
+            per[probe].append(a.elapsed_time(b) / 1e3 / blk)
+    t_plx_blk, t_soft_blk = statistics.median(per[True]), statistics.median(per[False])
+    t_soft = dist.max(t_soft_blk)
+    t_plx_blk = dist.max(t_plx_blk)
     rc, bits = ws.status()
     if rc != 0:
         raise SystemExit(f"device status after timing: {binding.parallax_status_string(rc)}")
 
-    # ---- per-kernel duration of the split-KV kernel (phase 1), live ----
-    nprof = min(args.steps, 1000 if use_graphs else 50)
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(nprof)]
-    for i in range(3):
-        step(bufs[i % nbuf])
-    torch.cuda.synchronize()
-    torch.cuda._sleep(int(4e8))  # let the host queue the launches ahead of the GPU
-    for i, (a, b) in enumerate(evs):
-        bb = bufs[i % nbuf]
-        a.record(stream)
-        binding.parallax_decode_phase(1, True, bb["q"], bb["r"], bb["k"], bb["v"], bb["seqlens"],
-                                      out, ws, scale=bb["scale"], num_splits=P, stream=stream)
-        b.record(stream)
-        binding.parallax_decode_phase(2, True, bb["q"], bb["r"], bb["k"], bb["v"], bb["seqlens"],
-                                      out, ws, scale=bb["scale"], num_splits=P, stream=stream)
-    torch.cuda.synchronize()
-    main_s = statistics.mean(a.elapsed_time(b) for a, b in evs) / 1e3
+    # ---- per-launch duration of the split-KV kernel (phase 1 only), live ----
+    # Back-to-back phase-1 launches (each waits for the previous one's end, so
+    # the period is one launch's duration). Launch-bound sizes replay them from
+    # a CUDA graph; large ones are timed with events around each launch.
+    def phase1(b):
+        binding.parallax_decode_phase(1, True, b["q"], b["r"], b["k"], b["v"], b["seqlens"],
+                                      out, ws, scale=b["scale"], num_splits=P, stream=stream)
+
+    if use_graphs:
+        g1 = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g1, stream=stream):
+            for b in bufs:
+                phase1(b)
+        reps = max(1, min(args.steps, 20000) // nbuf)
+        for _ in range(3):
+            g1.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(reps):
+            g1.replay()
+        e1.record(stream)
+        e1.synchronize()
+        main_s = e0.elapsed_time(e1) / 1e3 / (reps * nbuf)
+        main_launches = reps * nbuf
+    else:
+        nprof = min(args.steps, 50)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(nprof)]
+        for i, (a, b) in enumerate(evs):
+            a.record(stream)
+            phase1(bufs[i % nbuf])
+            b.record(stream)
+        torch.cuda.synchronize()
+        main_s = statistics.mean(a.elapsed_time(b) for a, b in evs) / 1e3
+        main_launches = nprof
+    step(bufs[0])  # leave a complete result behind
 
     # ---- end to end through the public API with host buffers ----
     pin = {k: x[k].cpu().pin_memory() for k in ("q", "r", "seqlens")}
@@ -428,7 +473,7 @@ def main():
 
     hbm_peak, peak_src = measured_peaks()
     N = dist.world
-    gbs = N * args.steps * step_kv / t_plx / 1e9
+    gbs = replicas.whole_job_rate(args.steps * step_kv, t_plx, N) / 1e9
     main_bytes = step_kv + qro_bytes(x)
     achieved = main_bytes / main_s / 1e9
     clocks = sampler.summary()
@@ -442,18 +487,20 @@ def main():
                    "num_splits": P, "l2": l2_note, "cuda_graphs": use_graphs},
         "us_per_step": t_plx / args.steps * 1e6,
         "kv_gbs_frac_of_hbm_peak": gbs / N / hbm_peak,
-        "softmax_r0": {"us_per_step": t_soft / args.steps * 1e6,
-                       "kv_gbs": N * args.steps * step_kv / t_soft / 1e9,
-                       "parallax_over_softmax_latency": t_plx / t_soft},
+        "softmax_r0": {"us_per_step": t_soft * 1e6, "kv_gbs": N * step_kv / t_soft / 1e9,
+                       "parallax_us_per_step_same_blocks": t_plx_blk * 1e6,
+                       "parallax_over_softmax_latency": t_plx_blk / t_soft,
+                       "method": f"{rounds} alternating blocks of {blk} steps each, medians"},
         "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons", "samples")},
         "e2e": {"value": N * k_e2e * step_kv / t_e2e / 1e9, "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "us_per_step": t_e2e / k_e2e * 1e6},
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": 2 * args.steps,  # split-KV + merge per step, in the timed region
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak, "traffic": profiled_traffic(),
                      "kernel": "parallax_tc_kernel (split-KV)", "peak_source": peak_src,
-                     "kernel_us": main_s * 1e6, "algorithmic_bytes_per_launch": main_bytes},
+                     "kernel_us": main_s * 1e6, "launches_timed": main_launches,
+                     "algorithmic_bytes_per_launch": main_bytes},
         "cpu_baseline": cpu,
     }
     if dist.rank == 0:

@@ -11,6 +11,7 @@
 #include <mutex>
 
 #include "parallax.h"
+#include "parallax_testing.h"
 
 #include "common.cuh"
 #include "kernel_generic.cuh"
@@ -377,6 +378,21 @@ const char* parallax_status_string(int status) {
 }
 
 }  // extern "C"
+
+extern "C" int parallax_testing_decode_stalled(const void* q, const void* r, const void* k_cache,
+                                               const void* v_cache, const int32_t* cache_seqlens,
+                                               void* out, int B, int Hq, int Hkv, int D,
+                                               float scale, void* stream, int Lmax,
+                                               int num_splits, void* workspace,
+                                               size_t workspace_bytes, int timeout_ms) {
+  if (timeout_ms < 1 || timeout_ms > 10000) return PARALLAX_ERR_BAD_SHAPE;
+  Call c = make_call(3, true, q, r, k_cache, v_cache, cache_seqlens, out, B, Hq, Hkv, D, scale,
+                     stream, Lmax, PARALLAX_DTYPE_BF16, PARALLAX_DTYPE_BF16, num_splits, workspace,
+                     workspace_bytes);
+  c.timeout_ns = (unsigned long long)timeout_ms * 1000000ull;
+  c.debug_skip_first_tile = 1;
+  return run(c);
+}
 
 // --------------------------------------------------------------------------
 // parallax_decode_noalloc: the same decode for callers that cannot allocate

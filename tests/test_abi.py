@@ -8,7 +8,9 @@ import pytest
 
 from parameterized_local_linear_b200 import binding, build
 
-HEADER = os.path.join(os.path.dirname(build.PKG), "include", "parallax.h")
+INCLUDE = os.path.join(os.path.dirname(build.PKG), "include")
+HEADER = os.path.join(INCLUDE, "parallax.h")
+HEADERS = sorted(os.path.join(INCLUDE, f) for f in os.listdir(INCLUDE) if f.endswith(".h"))
 
 OK, ENULL, ESHAPE, EHEAD, EDTYPE, EALIGN, EWS, ESPLITS = 0, -1, -2, -3, -4, -5, -6, -7
 
@@ -20,9 +22,11 @@ def lib():
 
 
 def declared_functions():
-    text = open(HEADER).read()
-    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(parallax_\w+)\s*\(", text)))
+    names = set()
+    for h in HEADERS:
+        text = re.sub(r"/\*.*?\*/", "", open(h).read(), flags=re.S)
+        names |= set(re.findall(r"\b(parallax_\w+)\s*\(", text))
+    return sorted(names)
 
 
 def test_header_declares_the_boundary():
@@ -40,7 +44,8 @@ def test_library_exports_every_declared_symbol(lib):
 
 def test_header_compiles_as_c(tmp_path):
     src = tmp_path / "t.c"
-    src.write_text('#include "parallax.h"\nint main(void){return PARALLAX_OK;}\n')
+    src.write_text("".join(f'#include "{os.path.basename(h)}"\n' for h in HEADERS) +
+                   "int main(void){return PARALLAX_OK;}\n")
     import subprocess
     subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.dirname(HEADER),
                     "-c", str(src), "-o", str(tmp_path / "t.o")], check=True)
@@ -105,6 +110,16 @@ def test_softmax_decode_does_not_need_r(lib):
     rc = lib.parallax_softmax_decode(16, 16, 16, 16, 16, 1, 16, 8, 128, ctypes.c_float(0.1),
                                      None, 64, 0, 0, 4, 16, 100)
     assert rc == EWS  # got past the pointer checks without r
+
+
+def test_stall_hook_rejects_bad_timeout(lib):
+    fn = lib.parallax_testing_decode_stalled
+    fn.argtypes = [ctypes.c_void_p] * 6 + [ctypes.c_int] * 4 + [ctypes.c_float, ctypes.c_void_p,
+                                                                ctypes.c_int, ctypes.c_int,
+                                                                ctypes.c_void_p, ctypes.c_size_t,
+                                                                ctypes.c_int]
+    assert fn(16, 16, 16, 16, 16, 16, 1, 16, 8, 128, 0.1, None, 64, 4, 16, 1 << 20, 0) == ESHAPE
+    assert fn(16, 16, 16, 16, 16, 16, 1, 16, 8, 128, 0.1, None, 64, 4, 16, 1 << 20, 20000) == ESHAPE
 
 
 def test_phase_selector(lib):

@@ -1,0 +1,51 @@
+"""Failure detection without a GPU fault: the split-KV kernel's waits are
+bounded. A testing hook tells the producer never to fill a CTA's first
+pipeline stage, so the consumers' wait on it runs out (50 ms here); the kernel
+must record PARALLAX_DEVICE_STATUS_TIMEOUT and return, and the same CUDA
+context must then run a normal decode correctly."""
+import ctypes
+import time
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parameterized_local_linear_b200 import binding, inputs
+
+pytestmark = pytest.mark.gpu
+
+TIMEOUT_BIT, ERR_DEVICE_TIMEOUT = 1, -9
+
+
+def test_bounded_wait_gives_up_and_context_survives():
+    assert torch.cuda.is_available()
+    lib = binding.load_library()
+    fn = lib.parallax_testing_decode_stalled
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    fn.argtypes = [vp] * 6 + [i] * 4 + [ctypes.c_float, vp, i, i, vp, ctypes.c_size_t, i]
+    fn.restype = i
+    w = inputs.custom_workload("stall", B=2, Hq=16, Hkv=8, D=128, Lmax=512, seed=31)
+    x = inputs.make_inputs(w, device="cuda")
+    ws = binding.Workspace(2, 16, 8, 128, 512, num_splits=4)
+    out = torch.empty((2, 16, 128), device="cuda", dtype=torch.bfloat16)
+    stream = torch.cuda.current_stream().cuda_stream
+    t0 = time.perf_counter()
+    rc = fn(x["q"].data_ptr(), x["r"].data_ptr(), x["k"].data_ptr(), x["v"].data_ptr(),
+            x["seqlens"].data_ptr(), out.data_ptr(), 2, 16, 8, 128, x["scale"], stream, 512, 4,
+            ws.ptr(), ws.nbytes, 50)
+    assert rc == 0
+    status, bits = ws.status(clear=True)  # synchronises
+    elapsed = time.perf_counter() - t0
+    assert bits & TIMEOUT_BIT and status == ERR_DEVICE_TIMEOUT
+    assert elapsed < 5.0, f"the stalled call took {elapsed:.2f} s"
+    assert ws.status() == (0, 0)
+
+    # the context is intact: a normal decode afterwards matches the oracle
+    got = binding.parallax_decode(x["q"], x["r"], x["k"], x["v"], x["seqlens"], scale=x["scale"],
+                                  out_dtype=torch.float32, num_splits=4, workspace=ws)
+    ref = oracle.parallax_decode(x["q"], x["r"], x["k"], x["v"], x["seqlens"], x["scale"])
+    g = got.double().cpu().numpy()
+    assert np.all(np.isfinite(g))
+    assert np.max(np.abs(g - ref) / np.maximum(1.0, np.abs(ref))) <= 1e-4
+    assert ws.status() == (0, 0)
