@@ -40,7 +40,9 @@ METRIC = "decode µs/step and KV-read GB/s (% of HBM peak) vs in-run R=0 softmax
 FALLBACK_HBM_GBS = 6650.0
 DEFAULT_STEPS = {"tiny": 20000, "qwen": 100000, "large": 200, "long": 200, "ragged": 200}
 DEFAULT_WARMUP = {"tiny": 2000, "qwen": 5000, "large": 5, "long": 5, "ragged": 5}
-MAIN_KERNEL_SRC = os.path.join(ROOT, "parameterized_local_linear_b200", "csrc", "kernel_tc.cuh")
+# the sources that decide what the split-KV kernel does (hashed against the ncu summary)
+MAIN_KERNEL_SRCS = [os.path.join(ROOT, "parameterized_local_linear_b200", "csrc", f)
+                    for f in ("kernel_tc.cuh", "partition.cuh", "common.cuh", "ptx.cuh")]
 
 
 def parse_args():
@@ -101,7 +103,10 @@ def profiled_traffic():
         text = open(path).read()
     except OSError:
         return None
-    src_hash = hashlib.sha256(open(MAIN_KERNEL_SRC, "rb").read()).hexdigest()[:16]
+    h = hashlib.sha256()
+    for f in MAIN_KERNEL_SRCS:
+        h.update(open(f, "rb").read())
+    src_hash = h.hexdigest()[:16]
     m_hash = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
     m_traffic = re.search(r"traffic_bytes_per_launch:\s*([0-9]+)", text)
     if not m_hash or not m_traffic or m_hash.group(1) != src_hash:

@@ -68,17 +68,14 @@ __host__ __device__ inline TcSmemLayout tc_smem_layout(int D, int stage_bytes, i
 }
 
 constexpr int kGenericThreads = 128;
-constexpr int kMergeThreads = 256;
-constexpr int kMergeMaxG = 128;        // query heads per kv head handled by the merge kernel
-constexpr int kMergeColsPerBlock = 32; // float4 columns of A/C one merge block sums
-constexpr int kMergeMaxPerThread = 4;  // records one thread loads in the one-pass merge
+constexpr int kMergeThreads = 128;  // one warp per SM sub-partition: fits beside a split-KV CTA
+constexpr int kMergeMaxG = 128;  // query heads per kv head handled by the merge kernel
+constexpr int kMergeChunk = 16;  // partial records one merge thread holds in registers
 
-// Merge blocks per partition: the owner's (head, 4-dim) output groups times
-// (A, C) are split so that each block sums about kMergeColsPerBlock float4
-// columns (never more than kMergeThreads).
+// Merge blocks per partition: one float4 column of A (and C) per thread.
 __host__ __device__ inline int merge_slices(int G, int D, bool probe) {
   const int cols = G * (D / 4) * (probe ? 2 : 1);
-  return (cols + kMergeColsPerBlock - 1) / kMergeColsPerBlock;
+  return (cols + kMergeThreads - 1) / kMergeThreads;
 }
 
 }  // namespace plx

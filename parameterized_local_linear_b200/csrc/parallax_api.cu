@@ -23,7 +23,7 @@ using namespace plx;
 namespace {
 
 constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;  // 2 s per wait
-constexpr long long kMinKeysPerSplit = 256;  // smallest key range worth a CTA
+constexpr long long kMinKeysPerSplit = 128;  // smallest key range worth a CTA (two tiles)
 constexpr int kCtasPerSm = 1;                // split-KV CTAs per SM (96 KB ring each)
 
 struct Call {

@@ -4,9 +4,9 @@
 // (b, g) holds n_b = clamp(cache_seqlens[b], 0, Lmax) keys and starts at
 // position Hkv * (n_0 + ... + n_{b-1}) + g * n_b. The P partitions (one CTA
 // each) cut this sequence of total = Hkv * sum_b n_b keys into equal ranges
-// [c*per, min((c+1)*per, total)), per = ceil(total / P), so every CTA streams
-// the same number of K/V bytes whatever the lengths (flash-decoding split-KV
-// with a balanced, length-aware cut). A range is processed as a series of
+// [c*per, min((c+1)*per, total)), per = ceil(total / P) rounded up to whole
+// 64-key tiles, so every CTA streams the same number of K/V bytes whatever the
+// lengths (flash-decoding split-KV with a balanced, length-aware cut). A range is processed as a series of
 // "pieces", the parts of the items it overlaps. A piece that is a whole item
 // is finished in place; any other piece writes a partial record to slot 2c
 // (the first piece of partition c) or 2c+1 (its last piece), and the
@@ -16,6 +16,8 @@
 #include <cstdint>
 
 namespace plx {
+
+constexpr int kRangeAlign = 64;  // partition ranges are multiples of one K/V tile
 
 __device__ __forceinline__ int clamp_len(int n, int Lmax) {
   return n < 0 ? 0 : (n > Lmax ? Lmax : n);
@@ -56,7 +58,9 @@ __device__ inline PartitionInfo locate_partition(const int32_t* __restrict__ seq
   PartitionInfo p;
   p.clamped = __any_sync(0xffffffffu, clamped);
   p.total = (long long)Hkv * __shfl_sync(0xffffffffu, incl, 31);
-  p.per = (p.total + P - 1) / P;
+  // ranges are whole 64-key tiles, so a range starts on a tile of its item
+  // whenever the items are tile multiples (trailing partitions may be empty)
+  p.per = ((p.total + P - 1) / P + kRangeAlign - 1) / kRangeAlign * kRangeAlign;
   p.lo = min(p.total, (long long)c * p.per);
   p.hi = min(p.total, p.lo + p.per);
   p.b = -1;

@@ -60,10 +60,11 @@ def test_status_strings(lib):
 
 def test_choose_splits_host_only(lib):
     # explicit SM count: pure host arithmetic
-    assert lib.parallax_choose_splits(1, 8, 4096, 148) == 128   # 32768 keys / 256
-    assert lib.parallax_choose_splits(2048, 8, 4096, 148) == 148  # one CTA per SM
+    assert lib.parallax_choose_splits(1, 8, 4096, 148) == 148     # one CTA per SM
+    assert lib.parallax_choose_splits(1, 8, 1024, 148) == 64      # 8192 keys / 128
+    assert lib.parallax_choose_splits(2048, 8, 4096, 148) == 148
     assert lib.parallax_choose_splits(1, 1, 1, 148) == 1
-    assert lib.parallax_choose_splits(2, 2, 128, 148) == 2  # 512 keys / 256
+    assert lib.parallax_choose_splits(2, 2, 128, 148) == 4  # 512 keys / 128
     assert lib.parallax_choose_splits(0, 8, 4096, 148) == ESHAPE
 
 
