@@ -29,9 +29,13 @@
  *    allocates no device memory and keeps no per-call state; the workspace is
  *    caller-owned scratch (see parallax_decode_workspace_bytes).
  *  - Layouts are contiguous, row-major, innermost last:
- *        q, r, out      [B][Hq][D]
- *        k_cache,v_cache[B][Hkv][Lmax][D]     (max-length-padded cache)
- *        cache_seqlens  [B] int32             (device memory)
+ *        q, r, out      [B][Hq][D]            (the pages' (B, 1, H, D))
+ *        k_cache,v_cache[B][Hkv][Lmax][D]     (max-length-padded cache;
+ *                       parallax_decode_ex also takes [B][Lmax][Hkv][D],
+ *                       the pages' (B, kv_len, H, D))
+ *        cache_seqlens  [B] int32 in device memory, or NULL: every sequence
+ *                       then holds all Lmax keys (the pages' call passes no
+ *                       lengths)
  *    Query head h reads kv head h / (Hq/Hkv) (contiguous GQA groups). Keys
  *    0 .. cache_seqlens[b]-1 of sequence b are attended; padding positions
  *    are never read into any accumulator. Values outside [0, Lmax] are
@@ -83,6 +87,10 @@ extern "C" {
 
 #define PARALLAX_MAX_SPLITS 65536
 
+/* Cache layouts for parallax_decode_ex. */
+#define PARALLAX_KV_BHSD 0 /* [B][Hkv][Lmax][D] */
+#define PARALLAX_KV_BSHD 1 /* [B][Lmax][Hkv][D] */
+
 /* Bits of the device status word kept at the start of the workspace. */
 #define PARALLAX_DEVICE_STATUS_TIMEOUT 1u
 #define PARALLAX_DEVICE_STATUS_SEQLEN_CLAMPED 2u
@@ -130,6 +138,30 @@ int parallax_softmax_decode(const void* q, const void* k_cache,
                             void* stream, int Lmax, int in_dtype, int out_dtype,
                             int num_splits, void* workspace,
                             size_t workspace_bytes);
+
+/*
+ * The general form of parallax_decode and parallax_softmax_decode.
+ *  - probe: 1 for the Parallax decode, 0 for the R = 0 softmax decode (r may
+ *    then be NULL).
+ *  - kv_layout: PARALLAX_KV_BHSD ([B][Hkv][Lmax][D], as parallax_decode) or
+ *    PARALLAX_KV_BSHD ([B][Lmax][Hkv][D], the cache layout of the
+ *    parallax-kernel 0.1.0 README, "Quickstart / Decoding (CuTeDSL)").
+ *  - window: 0 attends all cached keys; W > 0 attends only the last
+ *    min(n, W) keys of each sequence of length n (sliding-window decode; the
+ *    README's introduction calls sliding windows structurally compatible with
+ *    Parallax). The workspace size is that of Lmax = min(Lmax, W).
+ *  - phases: 3 runs both kernels; 1 or 2 runs only the split-KV or only the
+ *    merge kernel (as parallax_decode_phase).
+ * parallax_decode(...) is parallax_decode_ex(..., 1, PARALLAX_KV_BHSD, 0, 3).
+ * Errors as parallax_decode; a bad kv_layout or a negative window gives
+ * PARALLAX_ERR_BAD_SHAPE, a bad phases value PARALLAX_ERR_BAD_PHASE.
+ */
+int parallax_decode_ex(const void* q, const void* r, const void* k_cache,
+                       const void* v_cache, const int32_t* cache_seqlens, void* out,
+                       int B, int Hq, int Hkv, int D, float scale, void* stream,
+                       int Lmax, int in_dtype, int out_dtype, int num_splits,
+                       void* workspace, size_t workspace_bytes, int probe,
+                       int kv_layout, int window, int phases);
 
 /*
  * One phase of a decode call, for per-kernel timing and for tests of the

@@ -42,6 +42,7 @@ def load_library():
     lib.parallax_decode.argtypes = [vp, vp, vp, vp, vp, vp] + decode_tail
     lib.parallax_softmax_decode.argtypes = [vp, vp, vp, vp, vp] + decode_tail
     lib.parallax_decode_phase.argtypes = [i, i, vp, vp, vp, vp, vp, vp] + decode_tail
+    lib.parallax_decode_ex.argtypes = [vp, vp, vp, vp, vp, vp] + decode_tail + [i, i, i, i]
     lib.parallax_decode_workspace_bytes.argtypes = [i, i, i, i, i, i]
     lib.parallax_decode_workspace_bytes.restype = sz
     lib.parallax_choose_splits.argtypes = [i, i, i, i]
@@ -49,7 +50,8 @@ def load_library():
     lib.parallax_status_string.argtypes = [i]
     lib.parallax_status_string.restype = ctypes.c_char_p
     for fn in (lib.parallax_decode, lib.parallax_softmax_decode, lib.parallax_decode_phase,
-               lib.parallax_choose_splits, lib.parallax_workspace_status):
+               lib.parallax_decode_ex, lib.parallax_choose_splits,
+               lib.parallax_workspace_status):
         fn.restype = i
     _lib = lib
     return lib
@@ -104,36 +106,53 @@ def parallax_workspace_status(workspace: Workspace, clear: bool = False):
     return workspace.status(clear)
 
 
-def _shapes(q, k_cache, v_cache, cache_seqlens):
+KV_LAYOUTS = {"bhsd": 0, "bshd": 1}
+
+
+def _shapes(q, k_cache, v_cache, cache_seqlens, kv_layout="bhsd"):
     for name, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache),
                     ("cache_seqlens", cache_seqlens)):
+        if t is None and name == "cache_seqlens":
+            continue
         if not t.is_cuda:
             raise ValueError(f"{name} must be a CUDA tensor")
         if not t.is_contiguous():
             raise ValueError(f"{name} must be contiguous")
     if q.dim() != 3 or k_cache.dim() != 4 or v_cache.shape != k_cache.shape:
-        raise ValueError("expected q [B,Hq,D] and k_cache, v_cache [B,Hkv,Lmax,D]")
-    if cache_seqlens.dtype != torch.int32 or cache_seqlens.shape != (q.shape[0],):
+        raise ValueError("expected q [B,Hq,D] and a 4-D k_cache, v_cache")
+    if cache_seqlens is not None and (cache_seqlens.dtype != torch.int32
+                                      or cache_seqlens.shape != (q.shape[0],)):
         raise ValueError("cache_seqlens must be int32 [B]")
     if k_cache.dtype != q.dtype or v_cache.dtype != q.dtype or q.dtype not in _DTYPE_CODE:
         raise ValueError("q, r, k_cache, v_cache must share one dtype (bf16 or fp32)")
     B, Hq, D = q.shape
-    Bk, Hkv, Lmax, Dk = k_cache.shape
+    if kv_layout == "bshd":
+        Bk, Lmax, Hkv, Dk = k_cache.shape
+    elif kv_layout == "bhsd":
+        Bk, Hkv, Lmax, Dk = k_cache.shape
+    else:
+        raise ValueError("kv_layout must be 'bhsd' or 'bshd'")
     if Bk != B or Dk != D:
         raise ValueError("k_cache shape does not match q")
     return B, Hq, Hkv, D, Lmax
 
 
-def _prepare(q, k_cache, v_cache, cache_seqlens, out, out_dtype, workspace, num_splits):
-    B, Hq, Hkv, D, Lmax = _shapes(q, k_cache, v_cache, cache_seqlens)
+def _prepare(q, k_cache, v_cache, cache_seqlens, out, out_dtype, workspace, num_splits,
+             kv_layout="bhsd", window=0):
+    B, Hq, Hkv, D, Lmax = _shapes(q, k_cache, v_cache, cache_seqlens, kv_layout)
     if out is None:
         out = torch.empty((B, Hq, D), device=q.device,
                           dtype=out_dtype if out_dtype is not None else q.dtype)
     if out.shape != (B, Hq, D) or not out.is_contiguous() or out.dtype not in _DTYPE_CODE:
         raise ValueError("out must be a contiguous [B,Hq,D] bf16 or fp32 tensor")
     if workspace is None:
-        workspace = Workspace(B, Hq, Hkv, D, Lmax, num_splits, device=q.device)
+        eff = min(Lmax, window) if window > 0 else Lmax
+        workspace = Workspace(B, Hq, Hkv, D, eff, num_splits, device=q.device)
     return B, Hq, Hkv, D, Lmax, out, workspace
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
 
 
 def _stream(stream) -> int:
@@ -142,37 +161,80 @@ def _stream(stream) -> int:
     return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
 
 
-def parallax_decode(q, r, k_cache, v_cache, cache_seqlens, scale: Optional[float] = None,
+def parallax_decode(q, r, k_cache, v_cache, cache_seqlens=None, scale: Optional[float] = None,
                     out=None, out_dtype=None, num_splits: int = 0,
-                    workspace: Optional[Workspace] = None, stream=None):
-    """Parallax decode: out[b,h] = vbar + C/l - (b/l) vbar over the cached keys."""
+                    workspace: Optional[Workspace] = None, stream=None,
+                    kv_layout: Optional[str] = None, window: int = 0):
+    """Parallax decode: out[b,h] = vbar + C/l - (b/l) vbar over the cached keys.
+
+    q, r: [B, Hq, D], or the pages' (B, 1, Hq, D) (the cache layout then
+    defaults to (B, kv_len, Hkv, D) and the result has q's shape).
+    cache_seqlens: int32 [B], or None for full-length sequences.
+    kv_layout: 'bhsd' ([B, Hkv, Lmax, D], the default) or 'bshd'.
+    window: 0, or attend only the last `window` keys of each sequence."""
+    four_d = q.dim() == 4
+    if four_d:
+        if q.shape[1] != 1 or r.shape != q.shape:
+            raise ValueError("4-D q and r must be (B, 1, H, D)")
+        q, r = q.reshape(q.shape[0], q.shape[2], q.shape[3]), r.reshape(r.shape[0], r.shape[2], r.shape[3])
+    layout = kv_layout or ("bshd" if four_d else "bhsd")
     B, Hq, Hkv, D, Lmax, out, workspace = _prepare(q, k_cache, v_cache, cache_seqlens, out,
-                                                   out_dtype, workspace, num_splits)
+                                                   out_dtype, workspace, num_splits, layout,
+                                                   window)
     if r.shape != q.shape or r.dtype != q.dtype or not r.is_cuda or not r.is_contiguous():
         raise ValueError("r must be a contiguous CUDA tensor shaped like q")
     scale = D ** -0.5 if scale is None else scale
-    rc = load_library().parallax_decode(
-        q.data_ptr(), r.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
-        cache_seqlens.data_ptr(), out.data_ptr(), B, Hq, Hkv, D, float(scale),
-        _stream(stream), Lmax, _DTYPE_CODE[q.dtype], _DTYPE_CODE[out.dtype], int(num_splits),
-        workspace.ptr(), workspace.nbytes)
+    lib = load_library()
+    args = (q.data_ptr(), r.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+            _ptr(cache_seqlens), out.data_ptr(), B, Hq, Hkv, D, float(scale), _stream(stream),
+            Lmax, _DTYPE_CODE[q.dtype], _DTYPE_CODE[out.dtype], int(num_splits),
+            workspace.ptr(), workspace.nbytes)
+    if layout == "bhsd" and window == 0:
+        rc = lib.parallax_decode(*args)
+    else:
+        rc = lib.parallax_decode_ex(*args, 1, KV_LAYOUTS[layout], int(window), 3)
     _check(rc, "parallax_decode")
+    return out.reshape(B, 1, Hq, D) if four_d else out
+
+
+def parallax_softmax_decode(q, k_cache, v_cache, cache_seqlens=None,
+                            scale: Optional[float] = None, out=None, out_dtype=None,
+                            num_splits: int = 0, workspace: Optional[Workspace] = None,
+                            stream=None, kv_layout: str = "bhsd", window: int = 0):
+    """The R = 0 comparator: softmax attention decode on the same pipeline."""
+    B, Hq, Hkv, D, Lmax, out, workspace = _prepare(q, k_cache, v_cache, cache_seqlens, out,
+                                                   out_dtype, workspace, num_splits, kv_layout,
+                                                   window)
+    scale = D ** -0.5 if scale is None else scale
+    lib = load_library()
+    args = (q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), _ptr(cache_seqlens),
+            out.data_ptr(), B, Hq, Hkv, D, float(scale), _stream(stream), Lmax,
+            _DTYPE_CODE[q.dtype], _DTYPE_CODE[out.dtype], int(num_splits), workspace.ptr(),
+            workspace.nbytes)
+    if kv_layout == "bhsd" and window == 0:
+        rc = lib.parallax_softmax_decode(*args)
+    else:
+        rc = lib.parallax_decode_ex(args[0], None, *args[1:], 0, KV_LAYOUTS[kv_layout],
+                                    int(window), 3)
+    _check(rc, "parallax_softmax_decode")
     return out
 
 
-def parallax_softmax_decode(q, k_cache, v_cache, cache_seqlens, scale: Optional[float] = None,
-                            out=None, out_dtype=None, num_splits: int = 0,
-                            workspace: Optional[Workspace] = None, stream=None):
-    """The R = 0 comparator: softmax attention decode on the same pipeline."""
+def parallax_decode_ex(q, r, k_cache, v_cache, cache_seqlens, out, workspace: Workspace,
+                       scale: Optional[float] = None, num_splits: int = 0, probe: bool = True,
+                       kv_layout: str = "bhsd", window: int = 0, phases: int = 3, stream=None):
+    """The general entry point: probe (Parallax) or not (R = 0), either cache
+    layout, an optional sliding window, and the phases to run."""
     B, Hq, Hkv, D, Lmax, out, workspace = _prepare(q, k_cache, v_cache, cache_seqlens, out,
-                                                   out_dtype, workspace, num_splits)
+                                                   None, workspace, num_splits, kv_layout,
+                                                   window)
     scale = D ** -0.5 if scale is None else scale
-    rc = load_library().parallax_softmax_decode(
-        q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), cache_seqlens.data_ptr(),
-        out.data_ptr(), B, Hq, Hkv, D, float(scale), _stream(stream), Lmax,
+    rc = load_library().parallax_decode_ex(
+        q.data_ptr(), _ptr(r) if probe else None, k_cache.data_ptr(), v_cache.data_ptr(),
+        _ptr(cache_seqlens), out.data_ptr(), B, Hq, Hkv, D, float(scale), _stream(stream), Lmax,
         _DTYPE_CODE[q.dtype], _DTYPE_CODE[out.dtype], int(num_splits), workspace.ptr(),
-        workspace.nbytes)
-    _check(rc, "parallax_softmax_decode")
+        workspace.nbytes, int(bool(probe)), KV_LAYOUTS[kv_layout], int(window), int(phases))
+    _check(rc, "parallax_decode_ex")
     return out
 
 
@@ -185,7 +247,7 @@ def parallax_decode_phase(phase: int, probe: bool, q, r, k_cache, v_cache, cache
     scale = D ** -0.5 if scale is None else scale
     rc = load_library().parallax_decode_phase(
         int(phase), int(bool(probe)), q.data_ptr(), r.data_ptr() if r is not None else None,
-        k_cache.data_ptr(), v_cache.data_ptr(), cache_seqlens.data_ptr(), out.data_ptr(),
+        k_cache.data_ptr(), v_cache.data_ptr(), _ptr(cache_seqlens), out.data_ptr(),
         B, Hq, Hkv, D, float(scale), _stream(stream), Lmax, _DTYPE_CODE[q.dtype],
         _DTYPE_CODE[out.dtype], int(num_splits), workspace.ptr(), workspace.nbytes)
     _check(rc, "parallax_decode_phase")
@@ -210,7 +272,7 @@ def parallax_decode_noalloc(q, r, k_cache, v_cache, cache_seqlens, scale: Option
         raise ValueError("r must be a contiguous CUDA tensor shaped like q")
     scale = D ** -0.5 if scale is None else scale
     rc = fn(q.data_ptr(), r.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
-            cache_seqlens.data_ptr(), out.data_ptr(), B, Hq, Hkv, D, float(scale),
+            _ptr(cache_seqlens), out.data_ptr(), B, Hq, Hkv, D, float(scale),
             _stream(stream), Lmax, _DTYPE_CODE[q.dtype], _DTYPE_CODE[out.dtype], int(num_splits))
     _check(rc, "parallax_decode_noalloc")
     return out

@@ -17,9 +17,11 @@ __host__ __device__ constexpr int rec_floats(int D) { return kRecHead + 2 * D; }
 struct DecodeParams {
   const void* q;          // [B][Hq][D]
   const void* r;          // [B][Hq][D] (unused by the softmax kernels)
-  const void* k;          // [B][Hkv][Lmax][D] (generic kernel only; the TMA kernel uses tensor maps)
+  const void* k;          // K cache (generic kernel only; the TMA kernel uses tensor maps)
   const void* v;
-  const int32_t* seqlens; // [B]
+  long long kv_sb, kv_sh, kv_sk;  // element strides of batch row, kv head and key in K and V
+  const int32_t* seqlens; // [B], or NULL: every row holds Lmax keys
+  int window;             // > 0: attend only the last `window` keys of each row
   void* out;              // [B][Hq][D]
   float* partials;        // 2 * P * G records
   unsigned int* status;   // device status word (workspace header)

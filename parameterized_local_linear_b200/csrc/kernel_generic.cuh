@@ -40,7 +40,7 @@ __global__ void __launch_bounds__(kGenericThreads)
 
   pdl_wait_primary();  // launched with programmatic stream serialisation
   const PartitionInfo part =
-      locate_partition(p.seqlens, p.B, p.Hkv, p.Lmax, blockIdx.x, gridDim.x);
+      locate_partition(p.seqlens, p.B, p.Hkv, p.Lmax, p.window, blockIdx.x, gridDim.x);
   if (blockIdx.x == 0 && threadIdx.x == 0 && part.clamped) atomicOr(p.status, 2u);
   pdl_launch_dependents();
   if (part.lo >= part.hi) return;
@@ -52,19 +52,19 @@ __global__ void __launch_bounds__(kGenericThreads)
   const int tid = threadIdx.x, D = p.D, G = p.G, REC = rec_floats(D);
 
   PieceCursor cur;
-  cur.init(part, p.seqlens, p.B, p.Hkv, p.Lmax);
+  cur.init(part, p.seqlens, p.B, p.Hkv, p.Lmax, p.window);
   Piece pc;
   while (cur.next(pc)) {
-    const size_t item = (size_t)pc.b * p.Hkv + pc.g;
-    const T* kb = k + item * p.Lmax * D;
-    const T* vb = v + item * p.Lmax * D;
+    const long long kv0 = pc.b * p.kv_sb + pc.g * p.kv_sh + pc.kbase * p.kv_sk;
+    const T* kb = k + kv0;  // key j of the piece's item: kb + j * kv_sk
+    const T* vb = v + kv0;
     for (int h = 0; h < G; ++h) {
       const size_t row = ((size_t)pc.b * p.Hq + (size_t)pc.g * G + h) * D;
       float m = kNegInf, l = 0.f, bs = 0.f, A = 0.f, C = 0.f;
       for (int k0 = pc.i; k0 < pc.i + pc.len; k0 += kGenericThreads) {
         const int nk = min(kGenericThreads, pc.i + pc.len - k0);
         if (tid < nk) {
-          const T* kr = kb + (size_t)(k0 + tid) * D;
+          const T* kr = kb + (long long)(k0 + tid) * p.kv_sk;
           float t = 0.f, s = 0.f;
           for (int d = 0; d < D; ++d) {
             const float kd = to_f32(kr[d]);
@@ -88,7 +88,7 @@ __global__ void __launch_bounds__(kGenericThreads)
           l += e;
           if (PROBE) bs = fmaf(e, s_s[j], bs);
           if (tid < D) {
-            const float vd = to_f32(vb[(size_t)(k0 + j) * D + tid]);
+            const float vd = to_f32(vb[(long long)(k0 + j) * p.kv_sk + tid]);
             A = fmaf(e, vd, A);
             if (PROBE) C = fmaf(e * s_s[j], vd, C);
           }

@@ -41,12 +41,13 @@ __global__ void __launch_bounds__(kMergeThreads, 4) parallax_merge_kernel(const 
   const float kNegInf = __int_as_float(0xff800000u);
   const int tid = threadIdx.x;
   const int c = blockIdx.x, P = gridDim.x;
-  const PartitionInfo part = locate_partition(p.seqlens, p.B, p.Hkv, p.Lmax, c, P);
+  const PartitionInfo part = locate_partition(p.seqlens, p.B, p.Hkv, p.Lmax, p.window, c, P);
 
   // Sequences without keys: zero output (nothing else writes these rows).
   if (blockIdx.y == 0) {
     for (int b = c; b < p.B; b += P) {
-      if (clamp_len(__ldg(p.seqlens + b), p.Lmax) != 0) continue;
+      int kb;
+      if (attended_keys(p.seqlens, b, p.Lmax, p.window, &kb) != 0) continue;
       for (int idx = tid; idx < p.Hq * p.D; idx += kMergeThreads) {
         const size_t oi = (size_t)b * p.Hq * p.D + idx;
         if (OUT_F32)

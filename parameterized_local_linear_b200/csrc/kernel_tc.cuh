@@ -2,10 +2,10 @@
 //
 // One CTA per partition of the flattened key range (see partition.cuh),
 // persistent over the pieces of that range. Warp 4 is the producer: one lane
-// streams 64-key K and V tiles of the current item with one TMA each (4-D
-// tensor maps over the [B*Hkv][Lmax][D] caches, 128-byte swizzle, no
-// multicast) into a ring of shared-memory stages guarded by full/empty
-// mbarriers. Warps 0..3 consume: warp w owns keys 16w..16w+15 of every stage
+// streams 64-key K and V tiles of the current item with one TMA each (5-D
+// tensor maps {64 dims, keys, D/64 halves, kv heads, batch rows} over either
+// cache layout, 128-byte swizzle, no multicast) into a ring of shared-memory
+// stages guarded by full/empty mbarriers. Warps 0..3 consume: warp w owns keys 16w..16w+15 of every stage
 // and keeps its own online accumulators, so the consumer warps never
 // synchronise inside the key loop. They read the q (and r) rows of the item's
 // GQA group straight into mma fragments from global memory, overlapped with
@@ -86,7 +86,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // the previous kernel in the stream; nothing below may run before it ends.
   pdl_wait_primary();
   const PartitionInfo part =
-      locate_partition(p.seqlens, p.B, p.Hkv, p.Lmax, blockIdx.x, gridDim.x);
+      locate_partition(p.seqlens, p.B, p.Hkv, p.Lmax, p.window, blockIdx.x, gridDim.x);
   if (blockIdx.x == 0 && tid == 0 && part.clamped)
     atomicOr(p.status, 2u /* PARALLAX_DEVICE_STATUS_SEQLEN_CLAMPED */);
   // The merge grid may be scheduled once every CTA has its first stage in
@@ -100,13 +100,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (warp == kConsumerWarps) {
     if (lane != 0) return;
     PieceCursor cur;
-    cur.init(part, p.seqlens, p.B, p.Hkv, p.Lmax);
+    cur.init(part, p.seqlens, p.B, p.Hkv, p.Lmax, p.window);
     Piece pc;
     int stage = 0;
     uint32_t ph = 0, issued_mask = 0, issued_par = 0;
     bool ok = true, skip = p.debug_skip_first_tile != 0;
     while (ok && cur.next(pc)) {
-      const int item = pc.b * p.Hkv + pc.g;
       for (int k0 = pc.i; k0 < pc.i + pc.len; k0 += kTileKeys) {
         if (!mbar_wait_bounded(bar_empty + 8 * stage, ph ^ 1, p.timeout_ns, abort_flag)) {
           ok = false;
@@ -118,8 +117,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const uint32_t full = bar_full + 8 * stage;
           const uint32_t sK = base + stage * kStageBytes;
           mbar_arrive_expect_tx(full, kStageBytes);
-          tma_load_4d(sK, &tmK, 0, k0, 0, item, full, policy);
-          tma_load_4d(sK + kKBytes, &tmV, 0, k0, 0, item, full, policy);
+          const int key = pc.kbase + k0;  // cache position of the tile's first key
+          tma_load_5d(sK, &tmK, 0, key, 0, pc.g, pc.b, full, policy);
+          tma_load_5d(sK + kKBytes, &tmV, 0, key, 0, pc.g, pc.b, full, policy);
           if (issued_mask == 0) pdl_launch_dependents();
           issued_mask |= 1u << stage;
           issued_par = (issued_par & ~(1u << stage)) | (ph << stage);
@@ -160,7 +160,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int sw = lane & 7;  // row index mod 8 = the 128-byte swizzle phase of both rows
 
   PieceCursor cur;
-  cur.init(part, p.seqlens, p.B, p.Hkv, p.Lmax);
+  cur.init(part, p.seqlens, p.B, p.Hkv, p.Lmax, p.window);
   Piece pc;
   int stage = 0;
   uint32_t ph = 0, fph = 0;

@@ -38,6 +38,7 @@ struct Call {
   int Lmax, in_dtype, out_dtype, num_splits;
   void* ws;
   size_t ws_bytes;
+  int kv_layout, window;
   unsigned long long timeout_ns;
   int debug_skip_first_tile;
 };
@@ -80,6 +81,8 @@ size_t workspace_bytes_for(int G, int D, int P) {
   return kWorkspaceHeaderBytes + (size_t)2 * P * G * rec_floats(D) * sizeof(float);
 }
 
+int effective_len(int Lmax, int window) { return window > 0 && window < Lmax ? window : Lmax; }
+
 int resolve_splits(int num_splits, int B, int Hkv, int Lmax, int* P) {
   if (num_splits < 0 || num_splits > PARALLAX_MAX_SPLITS) return PARALLAX_ERR_BAD_SPLITS;
   if (num_splits > 0) {
@@ -94,9 +97,11 @@ int resolve_splits(int num_splits, int B, int Hkv, int Lmax, int* P) {
 }
 
 int validate(const Call& c) {
-  if (!c.q || !c.k || !c.v || !c.seqlens || !c.out || !c.ws) return PARALLAX_ERR_NULL_POINTER;
+  if (!c.q || !c.k || !c.v || !c.out || !c.ws) return PARALLAX_ERR_NULL_POINTER;
   if (c.probe && !c.r) return PARALLAX_ERR_NULL_POINTER;
   if (!shape_ok(c.B, c.Hq, c.Hkv, c.D, c.Lmax)) return PARALLAX_ERR_BAD_SHAPE;
+  if ((c.kv_layout != PARALLAX_KV_BHSD && c.kv_layout != PARALLAX_KV_BSHD) || c.window < 0)
+    return PARALLAX_ERR_BAD_SHAPE;
   if (c.D != 64 && c.D != 128) return PARALLAX_ERR_UNSUPPORTED_HEAD_DIM;
   if ((c.in_dtype != PARALLAX_DTYPE_BF16 && c.in_dtype != PARALLAX_DTYPE_F32) ||
       (c.out_dtype != PARALLAX_DTYPE_BF16 && c.out_dtype != PARALLAX_DTYPE_F32))
@@ -124,17 +129,30 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// [B*Hkv][Lmax][D] bf16 cache viewed as {64 dims, Lmax keys, D/64 halves,
-// B*Hkv items}: one box of 64 keys x D dims lands as D/64 swizzled
+// Element strides of (batch row, kv head, key) in a cache of either layout.
+struct KvStrides {
+  long long b, h, k;
+};
+KvStrides kv_strides(int layout, int Hkv, int Lmax, int D) {
+  if (layout == PARALLAX_KV_BSHD)
+    return {(long long)Lmax * Hkv * D, (long long)D, (long long)Hkv * D};
+  return {(long long)Hkv * Lmax * D, (long long)Lmax * D, (long long)D};
+}
+
+// A bf16 cache of either layout viewed as {64 dims, Lmax keys, D/64 halves,
+// Hkv heads, B rows}: one box of 64 keys x D dims lands as D/64 swizzled
 // [64 keys][128 bytes] blocks, one per 64-dim half.
-int encode_cache_map(CUtensorMap* map, const void* cache, int D, int Lmax, long long items) {
+int encode_cache_map(CUtensorMap* map, const void* cache, int D, int Lmax, int Hkv, int B,
+                     int layout) {
   auto enc = tensor_map_encoder();
   if (!enc) return PARALLAX_ERR_CUDA;
-  cuuint64_t dims[4] = {64, (cuuint64_t)Lmax, (cuuint64_t)(D / 64), (cuuint64_t)items};
-  cuuint64_t strides[3] = {(cuuint64_t)D * 2, 128, (cuuint64_t)Lmax * D * 2};
-  cuuint32_t box[4] = {64, (cuuint32_t)kTileKeys, (cuuint32_t)(D / 64), 1};
-  cuuint32_t elem[4] = {1, 1, 1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(cache), dims,
+  const KvStrides st = kv_strides(layout, Hkv, Lmax, D);
+  cuuint64_t dims[5] = {64, (cuuint64_t)Lmax, (cuuint64_t)(D / 64), (cuuint64_t)Hkv,
+                        (cuuint64_t)B};
+  cuuint64_t strides[4] = {(cuuint64_t)st.k * 2, 128, (cuuint64_t)st.h * 2, (cuuint64_t)st.b * 2};
+  cuuint32_t box[5] = {64, (cuuint32_t)kTileKeys, (cuuint32_t)(D / 64), 1, 1};
+  cuuint32_t elem[5] = {1, 1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(cache), dims,
                    strides, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? PARALLAX_OK : PARALLAX_ERR_CUDA;
@@ -165,9 +183,10 @@ int launch_tc(const Call& c, const DecodeParams& prm, int P) {
   int st = set_smem_once(kernel, L.total, done);
   if (st != PARALLAX_OK) return st;
   CUtensorMap tmK, tmV;
-  const long long items = (long long)c.B * c.Hkv;
-  if ((st = encode_cache_map(&tmK, c.k, D, c.Lmax, items)) != PARALLAX_OK) return st;
-  if ((st = encode_cache_map(&tmV, c.v, D, c.Lmax, items)) != PARALLAX_OK) return st;
+  if ((st = encode_cache_map(&tmK, c.k, D, c.Lmax, c.Hkv, c.B, c.kv_layout)) != PARALLAX_OK)
+    return st;
+  if ((st = encode_cache_map(&tmV, c.v, D, c.Lmax, c.Hkv, c.B, c.kv_layout)) != PARALLAX_OK)
+    return st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
@@ -239,7 +258,9 @@ int run(const Call& c) {
   int st = validate(c);
   if (st != PARALLAX_OK) return st;
   int P = 0;
-  if ((st = resolve_splits(c.num_splits, c.B, c.Hkv, c.Lmax, &P)) != PARALLAX_OK) return st;
+  if ((st = resolve_splits(c.num_splits, c.B, c.Hkv, effective_len(c.Lmax, c.window), &P)) !=
+      PARALLAX_OK)
+    return st;
   const int G = c.Hq / c.Hkv;
   if (c.ws_bytes < workspace_bytes_for(G, c.D, P)) return PARALLAX_ERR_WORKSPACE_TOO_SMALL;
 
@@ -248,7 +269,12 @@ int run(const Call& c) {
   prm.r = c.probe ? c.r : nullptr;
   prm.k = c.k;
   prm.v = c.v;
+  const KvStrides kst = kv_strides(c.kv_layout, c.Hkv, c.Lmax, c.D);
+  prm.kv_sb = kst.b;
+  prm.kv_sh = kst.h;
+  prm.kv_sk = kst.k;
   prm.seqlens = c.seqlens;
+  prm.window = c.window;
   prm.out = c.out;
   prm.status = static_cast<unsigned int*>(c.ws);
   prm.partials = reinterpret_cast<float*>(static_cast<char*>(c.ws) + kWorkspaceHeaderBytes);
@@ -292,6 +318,8 @@ Call make_call(int phases, bool probe, const void* q, const void* r, const void*
   c.num_splits = num_splits;
   c.ws = ws;
   c.ws_bytes = ws_bytes;
+  c.kv_layout = PARALLAX_KV_BHSD;
+  c.window = 0;
   c.timeout_ns = kDefaultTimeoutNs;
   c.debug_skip_first_tile = 0;
   return c;
@@ -332,6 +360,20 @@ int parallax_softmax_decode(const void* q, const void* k_cache, const void* v_ca
   return run(make_call(3, false, q, nullptr, k_cache, v_cache, cache_seqlens, out, B, Hq, Hkv, D,
                        scale, stream, Lmax, in_dtype, out_dtype, num_splits, workspace,
                        workspace_bytes));
+}
+
+int parallax_decode_ex(const void* q, const void* r, const void* k_cache, const void* v_cache,
+                       const int32_t* cache_seqlens, void* out, int B, int Hq, int Hkv, int D,
+                       float scale, void* stream, int Lmax, int in_dtype, int out_dtype,
+                       int num_splits, void* workspace, size_t workspace_bytes, int probe,
+                       int kv_layout, int window, int phases) {
+  if (phases < 1 || phases > 3) return PARALLAX_ERR_BAD_PHASE;
+  Call c = make_call(phases, probe != 0, q, r, k_cache, v_cache, cache_seqlens, out, B, Hq, Hkv,
+                     D, scale, stream, Lmax, in_dtype, out_dtype, num_splits, workspace,
+                     workspace_bytes);
+  c.kv_layout = kv_layout;
+  c.window = window;
+  return run(c);
 }
 
 int parallax_decode_phase(int phase, int probe, const void* q, const void* r, const void* k_cache,

@@ -23,12 +23,25 @@ __device__ __forceinline__ int clamp_len(int n, int Lmax) {
   return n < 0 ? 0 : (n > Lmax ? Lmax : n);
 }
 
+// The attended keys of batch row b: its clamped length n (every row holds Lmax
+// keys when there is no length array), and with a sliding window of W > 0
+// only the last min(n, W) of them. Returns that count; *kbase gets the first
+// attended key, n - count.
+__device__ __forceinline__ int attended_keys(const int32_t* __restrict__ seqlens, int b, int Lmax,
+                                             int window, int* kbase) {
+  const int n = seqlens ? clamp_len(__ldg(seqlens + b), Lmax) : Lmax;
+  const int ne = (window > 0 && n > window) ? window : n;
+  *kbase = n - ne;
+  return ne;
+}
+
 struct PartitionInfo {
   long long total;  // keys over all items
   long long per;    // keys per partition
   long long lo, hi; // this partition's range
   int b, g, i;      // item and key offset at position lo (valid if lo < hi)
-  int n;            // clamped length of batch b
+  int n;            // attended keys of batch b
+  int kbase;        // first attended key of batch b
   int clamped;      // some cache_seqlens value was outside [0, Lmax]
 };
 
@@ -38,16 +51,18 @@ struct PartitionInfo {
 // gives the prefix sums, and the lane whose chunk holds position lo walks it
 // to find the item there. c is this block's index among P partitions.
 __device__ inline PartitionInfo locate_partition(const int32_t* __restrict__ seqlens, int B,
-                                                 int Hkv, int Lmax, int c, int P) {
+                                                 int Hkv, int Lmax, int window, int c, int P) {
   const int lane = threadIdx.x & 31;
   const int chunk = (B + 31) / 32;
   const int b0 = min(B, lane * chunk), b1 = min(B, b0 + chunk);
   long long local = 0;
-  int clamped = 0;
+  int clamped = 0, kb;
   for (int b = b0; b < b1; ++b) {
-    const int n = __ldg(seqlens + b);
-    clamped |= (n < 0 || n > Lmax);
-    local += clamp_len(n, Lmax);
+    if (seqlens) {
+      const int n = __ldg(seqlens + b);
+      clamped |= (n < 0 || n > Lmax);
+    }
+    local += attended_keys(seqlens, b, Lmax, window, &kb);
   }
   long long incl = local;  // inclusive scan over lanes
 #pragma unroll
@@ -64,18 +79,19 @@ __device__ inline PartitionInfo locate_partition(const int32_t* __restrict__ seq
   p.lo = min(p.total, (long long)c * p.per);
   p.hi = min(p.total, p.lo + p.per);
   p.b = -1;
-  p.g = p.i = p.n = 0;
+  p.g = p.i = p.n = p.kbase = 0;
   // the lane whose batches contain position lo finds the item there
   long long pos = (long long)Hkv * (incl - local);
-  int fb = -1, fn = 0;
+  int fb = -1, fn = 0, fk = 0;
   long long within = 0;
   if (p.lo < p.hi && p.lo >= pos && p.lo < pos + (long long)Hkv * local) {
     for (int b = b0; b < b1; ++b) {
-      const int n = clamp_len(__ldg(seqlens + b), Lmax);
+      const int n = attended_keys(seqlens, b, Lmax, window, &kb);
       const long long blk = (long long)Hkv * n;
       if (p.lo < pos + blk) {
         fb = b;
         fn = n;
+        fk = kb;
         within = p.lo - pos;
         break;
       }
@@ -87,6 +103,7 @@ __device__ inline PartitionInfo locate_partition(const int32_t* __restrict__ seq
     const int src = __ffs(owner) - 1;
     p.b = __shfl_sync(0xffffffffu, fb, src);
     p.n = __shfl_sync(0xffffffffu, fn, src);
+    p.kbase = __shfl_sync(0xffffffffu, fk, src);
     const int w = (int)__shfl_sync(0xffffffffu, within, src);  // < Hkv * n <= Hkv * Lmax
     p.g = w / p.n;
     p.i = w - p.g * p.n;
@@ -96,24 +113,27 @@ __device__ inline PartitionInfo locate_partition(const int32_t* __restrict__ seq
 
 struct Piece {
   int b, g;      // item
-  int i, len;    // keys [i, i+len) of the item
-  int n;         // item length
+  int i, len;    // keys [i, i+len) of the item's attended range
+  int n;         // attended keys of the item
+  int kbase;     // cache position of the item's first attended key
   bool complete; // the piece is the whole item
   bool first;    // the first piece of this partition
 };
 
 // Walks the pieces of one partition; every role of a CTA walks the same list.
 struct PieceCursor {
-  int b, g, i, n;  // n: clamped length of batch b
+  int b, g, i, n, kbase;  // n, kbase: attended keys of batch b and the first one
   long long pos, lo, hi;
   const int32_t* seqlens;
-  int B, Hkv, Lmax;
+  int B, Hkv, Lmax, window;
 
-  __device__ void init(const PartitionInfo& p, const int32_t* sl, int B_, int Hkv_, int Lmax_) {
+  __device__ void init(const PartitionInfo& p, const int32_t* sl, int B_, int Hkv_, int Lmax_,
+                       int window_) {
     b = p.b;
     g = p.g;
     i = p.i;
     n = p.n;
+    kbase = p.kbase;
     pos = p.lo;
     lo = p.lo;
     hi = p.hi;
@@ -121,6 +141,7 @@ struct PieceCursor {
     B = B_;
     Hkv = Hkv_;
     Lmax = Lmax_;
+    window = window_;
   }
 
   __device__ bool next(Piece& pc) {
@@ -132,6 +153,7 @@ struct PieceCursor {
     pc.i = i;
     pc.len = len;
     pc.n = n;
+    pc.kbase = kbase;
     pc.complete = (i == 0) && (len == n);
     pc.first = (pos == lo);
     pos += len;
@@ -142,7 +164,7 @@ struct PieceCursor {
         g = 0;
         ++b;
         n = 0;
-        while (pos < hi && b < B && (n = clamp_len(__ldg(seqlens + b), Lmax)) == 0) ++b;
+        while (pos < hi && b < B && (n = attended_keys(seqlens, b, Lmax, window, &kbase)) == 0) ++b;
       }
     }
     return true;
