@@ -43,6 +43,8 @@ class Oracle:
         lib.oracle_parallax_expanded.argtypes = [dp, dp, dp, dp, ip, i, i, i, i, i, d, dp]
         lib.oracle_parallax_streaming.argtypes = [dp, dp, dp, dp, ip, i, i, i, i, i, d, i, dp]
         lib.oracle_softmax_decode.argtypes = [dp, dp, dp, ip, i, i, i, i, i, d, dp]
+        lib.oracle_parallax_prefill.argtypes = [dp, dp, dp, dp, i, i, i, i, i, d, i, dp]
+        lib.oracle_parallax_prefill.restype = ctypes.c_int
         for f in (lib.oracle_parallax_covariance, lib.oracle_parallax_expanded,
                   lib.oracle_parallax_streaming, lib.oracle_softmax_decode,
                   lib.oracle_num_threads):
@@ -106,6 +108,22 @@ class Oracle:
         self._check(rc, "oracle_softmax_decode")
         return out
 
+    def parallax_prefill(self, q, r, k, v, scale, causal=True):
+        """Training-shape forward: q, r [B, Hq, L, D], k, v [B, Hkv, L, D];
+        row i attends keys 0..i (all keys when causal is False)."""
+        q, r, k, v = _f64(q), _f64(r), _f64(k), _f64(v)
+        if q.ndim != 4 or r.shape != q.shape or k.ndim != 4 or v.shape != k.shape:
+            raise ValueError("expected q, r [B,Hq,L,D] and k, v [B,Hkv,L,D]")
+        B, Hq, L, D = q.shape
+        if k.shape[0] != B or k.shape[2] != L or k.shape[3] != D:
+            raise ValueError("shape mismatch between q and k")
+        out = np.zeros_like(q)
+        rc = self._lib.oracle_parallax_prefill(_ptr(q), _ptr(r), _ptr(k), _ptr(v), B, Hq,
+                                               k.shape[1], L, D, float(scale), int(bool(causal)),
+                                               _ptr(out))
+        self._check(rc, "oracle_parallax_prefill")
+        return out
+
     # The default used by parity checks: the definition (covariance) form.
     def parallax_decode(self, q, r, k, v, seqlens, scale):
         return self.parallax_covariance(q, r, k, v, seqlens, scale)
@@ -142,6 +160,10 @@ def softmax_decode(*a, **kw):
 
 def parallax_decode(*a, **kw):
     return default().parallax_decode(*a, **kw)
+
+
+def parallax_prefill(*a, **kw):
+    return default().parallax_prefill(*a, **kw)
 
 
 def num_threads() -> int:

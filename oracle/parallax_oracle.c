@@ -43,7 +43,9 @@
  *                                 time with a running max, in chunks that are
  *                                 combined by the max-rescaling merge
  * plus oracle_softmax_decode, the R = 0 special case written as plain softmax
- * attention.
+ * attention, and oracle_parallax_prefill, the training-shape forward (every
+ * query row of a sequence, causal), which applies the definition form to the
+ * keys each row sees.
  *
  * Readings where the pages are silent (all documented in the design notes):
  *   - layouts: q, r, out are [B][Hq][D]; k, v are [B][Hkv][Lmax][D];
@@ -352,6 +354,57 @@ int oracle_softmax_decode(const double* q, const double* k, const double* v,
                           int Lmax, int D, double scale, double* out) {
     return run(FORM_SOFTMAX, q, NULL, k, v, seqlens, B, Hq, Hkv, Lmax, D, scale,
                1, out);
+}
+
+/* ---- prefill (training-shape forward) -----------------------------------
+ *
+ * parallax-kernel 0.1.0 README, "Training (Triton)": parallax_func(q, r, k, v)
+ * maps (B, H, L, D) tensors to (B, H, L, D), causal. Row i of head h is the
+ * decode output above over keys 0..i of kv head h / (Hq/Hkv) (all L keys when
+ * causal == 0). Layouts: q, r, out [B][Hq][L][D]; k, v [B][Hkv][L][D].
+ */
+int oracle_parallax_prefill(const double* q, const double* r, const double* k,
+                            const double* v, int B, int Hq, int Hkv, int L, int D,
+                            double scale, int causal, double* out) {
+    if (!q || !r || !k || !v || !out) return ORACLE_EBADARG;
+    if (B < 0 || Hq < 1 || Hkv < 1 || L < 0 || D < 1 || Hq % Hkv != 0) return ORACLE_EBADARG;
+    int G = Hq / Hkv;
+    long long rows = (long long)B * Hq * L;
+    int failed = 0;
+#pragma omp parallel
+    {
+        int nmax = L > 0 ? L : 1;
+        double* t = malloc(sizeof(double) * (size_t)nmax);
+        double* s = malloc(sizeof(double) * (size_t)nmax);
+        double* w = malloc(sizeof(double) * (size_t)nmax);
+        double* vb = malloc(sizeof(double) * (size_t)D);
+        if (!t || !s || !w || !vb) {
+#pragma omp atomic write
+            failed = 1;
+        }
+#pragma omp for schedule(dynamic, 16)
+        for (long long x = 0; x < rows; ++x) {
+            if (!t || !s || !w || !vb) continue;
+            int b = (int)(x / ((long long)Hq * L));
+            int h = (int)((x / L) % Hq);
+            int i = (int)(x % L);
+            size_t qo = (((size_t)b * Hq + h) * (size_t)L + (size_t)i) * (size_t)D;
+            size_t ko = ((size_t)b * Hkv + (size_t)(h / G)) * (size_t)L * (size_t)D;
+            head_view hv;
+            hv.q = q + qo;
+            hv.r = r + qo;
+            hv.k = k + ko;
+            hv.v = v + ko;
+            hv.o = out + qo;
+            hv.n = causal ? i + 1 : L;
+            head_covariance(&hv, D, scale, t, s, w, vb);
+        }
+        free(t);
+        free(s);
+        free(w);
+        free(vb);
+    }
+    return failed ? ORACLE_ENOMEM : ORACLE_OK;
 }
 
 int oracle_num_threads(void) {

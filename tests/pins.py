@@ -271,8 +271,83 @@ def pin_empty_sequence_is_zero(orc):
         assert np.all(np.isfinite(got[1])), f"finite ({form})"
 
 
+# ------------------------------------------------------------------ prefill --
+
+def rand_prefill(seed, B=2, Hq=4, Hkv=2, L=12, D=8, r_scale=0.5):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((B, Hq, L, D))
+    r = rng.standard_normal((B, Hq, L, D)) * r_scale
+    k = rng.standard_normal((B, Hkv, L, D))
+    v = rng.standard_normal((B, Hkv, L, D))
+    return q, r, k, v
+
+
+def torch_sdpa(q, k, v, scale, causal):
+    """torch's own scaled_dot_product_attention in fp64 (GQA by repetition)."""
+    q, k, v = (torch.from_numpy(np.asarray(x, dtype=np.float64)) for x in (q, k, v))
+    G = q.shape[1] // k.shape[1]
+    k = torch.repeat_interleave(k, G, dim=1)
+    v = torch.repeat_interleave(v, G, dim=1)
+    return torch.nn.functional.scaled_dot_product_attention(q, k, v, is_causal=causal,
+                                                            scale=scale).numpy()
+
+
+def pin_prefill_r_zero_is_sdpa(orc):
+    q, r, k, v = rand_prefill(20, B=2, Hq=6, Hkv=3, L=17, D=8)
+    for causal in (True, False):
+        got = orc.parallax_prefill(q, np.zeros_like(r), k, v, 0.4, causal)
+        close(got, torch_sdpa(q, k, v, 0.4, causal), 1e-12, f"prefill r=0 causal={causal}")
+
+
+def pin_prefill_first_row_and_causality(orc):
+    q, r, k, v = rand_prefill(21)
+    o = orc.parallax_prefill(q, r, k, v, 0.3)
+    close(o[:, :, 0], np.repeat(v[:, :, 0], 2, axis=1), 1e-12, "prefill row 0 = v_0")
+    # rows 0..5 must not depend on keys or values at positions 6..L-1
+    k2, v2 = k.copy(), v.copy()
+    k2[:, :, 6:] += 5.0 * np.random.default_rng(22).standard_normal(k2[:, :, 6:].shape)
+    v2[:, :, 6:] = np.nan
+    o2 = orc.parallax_prefill(q, r, k2, v2, 0.3)
+    close(o2[:, :, :6], o[:, :, :6], 1e-12, "prefill causality")
+
+
+def pin_prefill_local_linear_intercept(orc):
+    """Causal row i with r_i = Sigma_w^{-1}(q_i - kbar) is the WLS intercept
+    over keys 0..i (numpy lstsq), like the decode pin."""
+    rng = np.random.default_rng(23)
+    L, D, scale, i = 15, 4, 0.7, 13
+    q = rng.standard_normal((1, 1, L, D))
+    k = rng.standard_normal((1, 1, L, D))
+    v = rng.standard_normal((1, 1, L, D))
+    kk, vv, qi = k[0, 0, :i + 1], v[0, 0, :i + 1], q[0, 0, i]
+    t = scale * kk @ qi
+    w = np.exp(t - t.max())
+    w /= w.sum()
+    kbar = w @ kk
+    sigma = (kk - kbar).T @ ((kk - kbar) * w[:, None])
+    r = np.zeros_like(q)
+    r[0, 0, i] = np.linalg.solve(sigma, qi - kbar)
+    X = np.hstack([np.ones((i + 1, 1)), kk - qi])
+    sw = np.sqrt(w)[:, None]
+    coef, *_ = np.linalg.lstsq(X * sw, vv * sw, rcond=None)
+    close(orc.parallax_prefill(q, r, k, v, scale)[0, 0, i], coef[0], 1e-9, "prefill LLA intercept")
+
+
+def pin_prefill_gqa_mapping(orc):
+    q, r, k, v = rand_prefill(24, Hq=8, Hkv=2)
+    v[:, 0] = 1.0
+    v[:, 1] = 2.0
+    o = orc.parallax_prefill(q, r, k, v, 0.3)
+    want = np.zeros_like(o)
+    want[:, :4] = 1.0
+    want[:, 4:] = 2.0
+    close(o, want, 1e-12, "prefill GQA mapping")
+
+
 PINS = [pin_hand_examples, pin_r_zero_is_softmax, pin_single_key_returns_v,
         pin_constant_values, pin_value_shift_and_scale, pin_key_translation,
         pin_linear_in_r, pin_key_permutation, pin_forms_agree,
         pin_local_linear_intercept, pin_gqa_mapping, pin_lengths_exact,
-        pin_empty_sequence_is_zero]
+        pin_empty_sequence_is_zero, pin_prefill_r_zero_is_sdpa,
+        pin_prefill_first_row_and_causality, pin_prefill_local_linear_intercept,
+        pin_prefill_gqa_mapping]

@@ -42,6 +42,11 @@ MUTANTS = [
     ("b accumulates e", "a->b = alpha * a->b + e * s;", "a->b = alpha * a->b + e;"),
     ("softmax without normalisation", "for (int i = 0; i < n; ++i) w[i] /= z;",
      "for (int i = 0; i < n; ++i) w[i] /= 1.0;"),
+    ("prefill sees its own key only from row 1", "hv.n = causal ? i + 1 : L;",
+     "hv.n = causal ? (i > 0 ? i : 1) : L;"),
+    ("prefill GQA modulo mapping",
+     "size_t ko = ((size_t)b * Hkv + (size_t)(h / G)) * (size_t)L * (size_t)D;",
+     "size_t ko = ((size_t)b * Hkv + (size_t)(h % Hkv)) * (size_t)L * (size_t)D;"),
 ]
 
 
