@@ -180,6 +180,26 @@ int parallax_decode_phase(int phase, int probe, const void* q, const void* r,
                           void* workspace, size_t workspace_bytes);
 
 /*
+ * The training-shape (prefill) forward: parallax-kernel 0.1.0 README,
+ * "Training (Triton)": parallax_func(q, r, k, v) maps (B, H, L, D) to
+ * (B, H, L, D), causal. Row i of query head h is the decode output above over
+ * keys 0..i of kv head h / (Hq/Hkv) (all L keys when causal == 0).
+ *  - q, r, out [B][Hq][L][D]; k, v [B][Hkv][L][D]; bf16 inputs (device
+ *    pointers, 16-byte aligned); out bf16 or fp32 (out_dtype).
+ *  - D is 64 or 128; B and Hq at most 65535.
+ *  - The products Q K^T, R K^T, P V and (P o T) V run on the tcgen05 tensor
+ *    cores (operands in shared memory, accumulators in tensor memory); the
+ *    probabilities enter the value products as bf16 hi + lo pairs.
+ *  - workspace: at least 256 bytes, zeroed once; its first word is the device
+ *    status word read by parallax_workspace_status.
+ * Errors as parallax_decode.
+ */
+int parallax_prefill(const void* q, const void* r, const void* k, const void* v,
+                     void* out, int B, int Hq, int Hkv, int L, int D, float scale,
+                     int causal, void* stream, int out_dtype, void* workspace,
+                     size_t workspace_bytes);
+
+/*
  * Synchronise the current device, then read (and, if clear != 0, zero) the
  * device status word at the start of a workspace. *device_status receives PARALLAX_DEVICE_STATUS_* bits;
  * the return value maps them to a status: PARALLAX_ERR_DEVICE_TIMEOUT if a

@@ -276,3 +276,32 @@ def parallax_decode_noalloc(q, r, k_cache, v_cache, cache_seqlens, scale: Option
             _stream(stream), Lmax, _DTYPE_CODE[q.dtype], _DTYPE_CODE[out.dtype], int(num_splits))
     _check(rc, "parallax_decode_noalloc")
     return out
+
+
+def parallax_prefill(q, r, k, v, scale: Optional[float] = None, causal: bool = True, out=None,
+                     out_dtype=None, workspace=None, stream=None):
+    """Training-shape forward (the README's parallax_func): q, r [B, Hq, L, D],
+    k, v [B, Hkv, L, D] bf16 -> [B, Hq, L, D]; row i attends keys 0..i."""
+    lib = load_library()
+    fn = lib.parallax_prefill
+    vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    fn.argtypes = [vp] * 5 + [i] * 5 + [f, i, vp, i, vp, ctypes.c_size_t]
+    fn.restype = i
+    for name, t in (("q", q), ("r", r), ("k", k), ("v", v)):
+        if not t.is_cuda or not t.is_contiguous() or t.dtype != torch.bfloat16 or t.dim() != 4:
+            raise ValueError(f"{name} must be a contiguous 4-D bf16 CUDA tensor")
+    B, Hq, L, D = q.shape
+    if r.shape != q.shape or k.shape != v.shape or k.shape[0] != B or k.shape[2:] != (L, D):
+        raise ValueError("expected q, r [B, Hq, L, D] and k, v [B, Hkv, L, D]")
+    Hkv = k.shape[1]
+    if out is None:
+        out = torch.empty_like(q, dtype=out_dtype if out_dtype is not None else q.dtype)
+    if workspace is None:
+        workspace = torch.zeros(256, dtype=torch.uint8, device=q.device)
+    buf = workspace.buffer if isinstance(workspace, Workspace) else workspace
+    scale = D ** -0.5 if scale is None else scale
+    rc = fn(q.data_ptr(), r.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, Hq, Hkv,
+            L, D, float(scale), int(bool(causal)), _stream(stream), _DTYPE_CODE[out.dtype],
+            buf.data_ptr(), buf.numel())
+    _check(rc, "parallax_prefill")
+    return out

@@ -16,6 +16,7 @@
 #include "common.cuh"
 #include "kernel_generic.cuh"
 #include "kernel_merge.cuh"
+#include "kernel_prefill.cuh"
 #include "kernel_tc.cuh"
 
 using namespace plx;
@@ -420,6 +421,85 @@ const char* parallax_status_string(int status) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------- prefill ----
+namespace {
+
+// [rows_per_item * items][D] bf16 viewed as {64 dims, L rows, D/64 halves,
+// items}: one box of `box_rows` rows x D dims lands as D/64 swizzled
+// [box_rows][128 bytes] blocks (the UMMA operand layout).
+int encode_rows_map(CUtensorMap* map, const void* base, int D, int L, long long items,
+                    int box_rows) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return PARALLAX_ERR_CUDA;
+  cuuint64_t dims[4] = {64, (cuuint64_t)L, (cuuint64_t)(D / 64), (cuuint64_t)items};
+  cuuint64_t strides[3] = {(cuuint64_t)D * 2, 128, (cuuint64_t)L * D * 2};
+  cuuint32_t box[4] = {64, (cuuint32_t)box_rows, (cuuint32_t)(D / 64), 1};
+  cuuint32_t elem[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
+                   strides, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? PARALLAX_OK : PARALLAX_ERR_CUDA;
+}
+
+template <int D, bool OUT_F32>
+int launch_prefill(const void* q, const void* r, const void* k, const void* v,
+                   const PrefillParams& prm, int Hq, int Hkv, int L, int B,
+                   cudaStream_t stream) {
+  auto kernel = parallax_prefill_kernel<D, OUT_F32>;
+  static int done[256] = {0};
+  int st = set_smem_once(kernel, PfGeom<D>::kSmem, done);
+  if (st != PARALLAX_OK) return st;
+  CUtensorMap tq, tr, tk, tv;
+  if ((st = encode_rows_map(&tq, q, D, L, (long long)B * Hq, kPfRows)) != PARALLAX_OK) return st;
+  if ((st = encode_rows_map(&tr, r, D, L, (long long)B * Hq, kPfRows)) != PARALLAX_OK) return st;
+  if ((st = encode_rows_map(&tk, k, D, L, (long long)B * Hkv, kPfKeys)) != PARALLAX_OK) return st;
+  if ((st = encode_rows_map(&tv, v, D, L, (long long)B * Hkv, kPfKeys)) != PARALLAX_OK) return st;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)prm.num_qt, (unsigned)Hq, (unsigned)B);
+  cfg.blockDim = dim3(kPfThreads);
+  cfg.dynamicSmemBytes = PfGeom<D>::kSmem;
+  cfg.stream = stream;
+  return cudaLaunchKernelEx(&cfg, kernel, tq, tr, tk, tv, prm) == cudaSuccess ? PARALLAX_OK
+                                                                              : PARALLAX_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" int parallax_prefill(const void* q, const void* r, const void* k, const void* v,
+                                void* out, int B, int Hq, int Hkv, int L, int D, float scale,
+                                int causal, void* stream, int out_dtype, void* workspace,
+                                size_t workspace_bytes) {
+  if (!q || !r || !k || !v || !out || !workspace) return PARALLAX_ERR_NULL_POINTER;
+  if (B < 1 || Hq < 1 || Hkv < 1 || L < 1 || Hq % Hkv != 0 || B > 65535 || Hq > 65535)
+    return PARALLAX_ERR_BAD_SHAPE;
+  if (D != 64 && D != 128) return PARALLAX_ERR_UNSUPPORTED_HEAD_DIM;
+  if (out_dtype != PARALLAX_DTYPE_BF16 && out_dtype != PARALLAX_DTYPE_F32)
+    return PARALLAX_ERR_UNSUPPORTED_DTYPE;
+  if (!aligned16(q) || !aligned16(r) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+      !aligned16(workspace))
+    return PARALLAX_ERR_MISALIGNED;
+  if (workspace_bytes < kWorkspaceHeaderBytes) return PARALLAX_ERR_WORKSPACE_TOO_SMALL;
+  PrefillParams prm{};
+  prm.out = out;
+  prm.status = static_cast<unsigned int*>(workspace);
+  prm.B = B;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.G = Hq / Hkv;
+  prm.L = L;
+  prm.num_qt = (L + kPfRows - 1) / kPfRows;
+  prm.causal = causal != 0;
+  prm.scale_log2 = (float)((double)scale * 1.4426950408889634);
+  prm.timeout_ns = kDefaultTimeoutNs;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool f32 = out_dtype == PARALLAX_DTYPE_F32;
+  if (D == 128)
+    return f32 ? launch_prefill<128, true>(q, r, k, v, prm, Hq, Hkv, L, B, s)
+               : launch_prefill<128, false>(q, r, k, v, prm, Hq, Hkv, L, B, s);
+  return f32 ? launch_prefill<64, true>(q, r, k, v, prm, Hq, Hkv, L, B, s)
+             : launch_prefill<64, false>(q, r, k, v, prm, Hq, Hkv, L, B, s);
+}
 
 extern "C" int parallax_testing_decode_stalled(const void* q, const void* r, const void* k_cache,
                                                const void* v_cache, const int32_t* cache_seqlens,

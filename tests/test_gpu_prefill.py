@@ -1,0 +1,58 @@
+"""GPU parity of the tcgen05 prefill forward (the README's parallax_func,
+"Training (Triton)": (B, H, L, D) -> (B, H, L, D), causal) against the fp64
+oracle's prefill. Partial 128-row query tiles and 64-key tiles, GQA, both
+head dimensions, causal and not, bf16 and fp32 outputs."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parameterized_local_linear_b200 import binding
+
+pytestmark = pytest.mark.gpu
+
+TOL = {torch.bfloat16: 2e-2, torch.float32: 1e-4}
+
+
+def make(B, Hq, Hkv, L, D, seed, r_scale=0.5):
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    q = torch.randn(B, Hq, L, D, device="cuda", dtype=torch.bfloat16, generator=g)
+    r = (torch.randn(B, Hq, L, D, device="cuda", dtype=torch.bfloat16, generator=g) * r_scale).to(
+        torch.bfloat16)
+    k = torch.randn(B, Hkv, L, D, device="cuda", dtype=torch.bfloat16, generator=g)
+    v = torch.randn(B, Hkv, L, D, device="cuda", dtype=torch.bfloat16, generator=g)
+    return q, r, k, v
+
+
+def scaled_error(got, ref):
+    g = got.float().cpu().double().numpy()
+    assert np.all(np.isfinite(g)), "non-finite output"
+    return float(np.max(np.abs(g - ref) / np.maximum(1.0, np.abs(ref))))
+
+
+@pytest.mark.parametrize("L", [1, 64, 200, 384])
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("Hq,Hkv", [(2, 2), (4, 2)])
+def test_prefill_matches_oracle(L, D, Hq, Hkv):
+    q, r, k, v = make(2, Hq, Hkv, L, D, seed=300 + L + D + Hq)
+    scale = D ** -0.5
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    for causal in (True, False):
+        want = oracle.parallax_prefill(q, r, k, v, scale, causal)
+        for out_dtype in (torch.bfloat16, torch.float32):
+            got = binding.parallax_prefill(q, r, k, v, scale=scale, causal=causal,
+                                           out_dtype=out_dtype, workspace=ws)
+            err = scaled_error(got, want)
+            assert err <= TOL[out_dtype], (L, D, Hq, Hkv, causal, out_dtype, err)
+    torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32).item()) == 0  # no device timeout
+
+
+def test_prefill_r_zero_and_deterministic():
+    q, r, k, v = make(1, 4, 4, 300, 128, seed=320)
+    z = torch.zeros_like(r)
+    want = oracle.parallax_prefill(q, z, k, v, 128 ** -0.5, True)
+    a = binding.parallax_prefill(q, z, k, v, out_dtype=torch.float32)
+    b = binding.parallax_prefill(q, z, k, v, out_dtype=torch.float32)
+    assert torch.equal(a, b)
+    assert scaled_error(a, want) <= 1e-4
