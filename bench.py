@@ -3,6 +3,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload qwen|large|long|ragged|tiny]
     python bench.py --impl reference ...   # the fp64 CPU oracle as the reference arm
+    python bench.py --prefill [--prefill-shape B,Hq,Hkv,L,D]   # the causal training-shape forward
 
 A step is one Parallax decode pass (split-KV kernel + merge kernel) over one
 batch of synthetic input resident in HBM. The headline value is KV-read
@@ -37,7 +38,11 @@ sys.path.insert(0, ROOT)
 from parameterized_local_linear_b200 import inputs, replicas  # noqa: E402
 
 METRIC = "decode µs/step and KV-read GB/s (% of HBM peak) vs in-run R=0 softmax decode"
+PREFILL_METRIC = "prefill forward TFLOP/s (algorithmic, causal) vs in-run softmax attention"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+# Qwen-3-0.6B attention heads (16 query, 8 kv, D = 128) at a 4096-token context
+PREFILL_DEFAULT_SHAPE = "4,16,8,4096,128"
 DEFAULT_STEPS = {"tiny": 20000, "qwen": 100000, "large": 200, "long": 200, "ragged": 200}
 DEFAULT_WARMUP = {"tiny": 2000, "qwen": 5000, "large": 5, "long": 5, "ragged": 5}
 # the sources that decide what the split-KV kernel does (hashed against the ncu summary)
@@ -58,7 +63,14 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="bound of the CPU oracle baseline sample (seconds)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--prefill", action="store_true",
+                    help="time the causal training-shape forward instead of the decode")
+    ap.add_argument("--prefill-shape", default=PREFILL_DEFAULT_SHAPE,
+                    help="B,Hq,Hkv,L,D of the prefill forward")
     a = ap.parse_args()
+    if a.prefill:
+        a.steps = a.steps if a.steps is not None else 50
+        a.warmup = a.warmup if a.warmup is not None else 5
     a.steps = a.steps if a.steps is not None else DEFAULT_STEPS[a.workload]
     a.warmup = a.warmup if a.warmup is not None else DEFAULT_WARMUP[a.workload]
     return a
@@ -93,6 +105,17 @@ def measured_peaks():
         return float(d["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def measured_bf16_peak():
+    """Dense bf16 tensor peak: the burst figure (a kernel timed on its own)."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback"
 
 
 def profiled_traffic():
@@ -293,10 +316,196 @@ def run_reference(args):
     return 0
 
 
+# ------------------------------------------------------- prefill forward ----
+
+def prefill_flops(B, Hq, L, D, causal=True):
+    """Algorithmic flops of the forward: q.k, r.k, e.v and (e s).v, 2 D flops
+    each per (query head, row, attended key)."""
+    pairs = L * (L + 1) // 2 if causal else L * L
+    return 8 * D * B * Hq * pairs
+
+
+def prefill_inputs(B, Hq, Hkv, L, D, device, seed=7):
+    """The pages' quickstart recipe for the training shape: q, r, k, v all
+    bf16 N(0, 1) (parallax-kernel 0.1.0 README, "Training (Triton)")."""
+    g = torch.Generator(device=device).manual_seed(seed)
+    mk = lambda H: torch.randn(B, H, L, D, device=device, dtype=torch.bfloat16, generator=g)
+    return mk(Hq), mk(Hq), mk(Hkv), mk(Hkv)
+
+
+def prefill_oracle_sample(shape, budget_s):
+    """The fp64 oracle on the first query heads of batch row 0 (full length),
+    as many as fit in about budget_s. Returns (TFLOP/s, threads, description)."""
+    import oracle
+    B, Hq, Hkv, L, D = shape
+    G = Hq // Hkv
+    q, r, k, v = prefill_inputs(1, G, 1, L, D, "cpu")
+    t0 = time.perf_counter()
+    oracle.parallax_prefill(q[:, :1], r[:, :1], k, v, D ** -0.5, True)
+    one = max(1e-4, time.perf_counter() - t0)
+    heads = max(1, min(G, int(budget_s / one)))
+    reps = max(1, int(budget_s / (one * heads)))
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        oracle.parallax_prefill(q[:, :heads], r[:, :heads], k, v, D ** -0.5, True)
+    secs = time.perf_counter() - t0
+    tf = prefill_flops(1, heads, L, D) * reps / secs / 1e12
+    desc = (f"fp64 oracle prefill, {reps} passes over {heads} query head(s) of one batch row "
+            f"at L={L}, D={D}; {secs:.1f} s")
+    return tf, oracle.num_threads(), desc, secs
+
+
+def run_prefill(args):
+    """Causal training-shape forward: one step is one parallax_prefill launch
+    over the whole [B, H, L, D] problem, inputs resident in HBM."""
+    shape = tuple(int(t) for t in args.prefill_shape.split(","))
+    B, Hq, Hkv, L, D = shape
+    flops = prefill_flops(B, Hq, L, D)
+    cfg = {"workload": f"prefill: Parallax causal forward B={B} Hq={Hq} Hkv={Hkv} L={L} D={D} "
+                       f"bf16 N(0,1)", "global_batch": B, "seq_len": L}
+    if args.impl == "reference":
+        if int(os.environ.get("RANK", "0")) != 0:
+            return 0
+        tf, cores, desc, secs = prefill_oracle_sample(shape, min(10.0, args.cpu_seconds))
+        line = {"impl": "reference", "metric": PREFILL_METRIC, "value": tf, "unit": "TFLOP/s",
+                "n_gpus": args.gpus, "steps": 1, "warmup": 0, "ms_per_step": secs * 1e3,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "config": cfg,
+                "cpu_baseline": {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                                 "sample": desc},
+                "e2e": {"value": tf, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return 0
+
+    from parameterized_local_linear_b200 import binding
+    dist = Dist(args.gpus)
+    dist.init_gpu()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    binding.load_library()
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.set_stream(stream)
+    q, r, k, v = prefill_inputs(B, Hq, Hkv, L, D, dev)
+    out = torch.empty_like(q)
+    ws = torch.zeros(256, dtype=torch.uint8, device=dev)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    in_bytes = sum(t.numel() * t.element_size() for t in (q, r, k, v, out))
+    flush = torch.empty(2 * l2 // 4, dtype=torch.float32, device=dev) if in_bytes < 2 * l2 else None
+
+    def run(k_steps, events=None):
+        for i in range(k_steps):
+            if flush is not None:
+                flush.fill_(float(i))
+            if events:
+                events[i][0].record(stream)
+            binding.parallax_prefill(q, r, k, v, out=out, workspace=ws, stream=stream)
+            if events:
+                events[i][1].record(stream)
+
+    def timed(fn, k_steps, w_steps, sampler=None):
+        fn(w_steps)
+        torch.cuda.synchronize()
+        dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if sampler:
+            sampler.__enter__()
+        e0.record(stream)
+        fn(k_steps)
+        e1.record(stream)
+        e1.synchronize()
+        if sampler:
+            sampler.__exit__(None, None, None)
+        torch.cuda.synchronize()
+        dist.barrier()
+        return dist.max(e0.elapsed_time(e1) / 1e3)
+
+    sampler = ClockSampler(dev.index)
+    t_step = timed(run, args.steps, args.warmup, sampler)
+    # per-launch kernel duration (events around each launch; the L2 flush sits outside)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    run(args.steps, evs)
+    torch.cuda.synchronize()
+    kern_s = statistics.median(a.elapsed_time(b) for a, b in evs) / 1e3
+    st = int(ws[:4].view(torch.int32).item())
+    if st != 0:
+        raise SystemExit(f"device status after timing: {st:#x}")
+
+    # in-run softmax-only attention on the same q, k, v (torch SDPA, causal,
+    # grouped heads): context for the tensor-core efficiency, not the target
+    sdpa = None
+    try:
+        def run_sdpa(k_steps):
+            for i in range(k_steps):
+                if flush is not None:
+                    flush.fill_(float(i))
+                torch.nn.functional.scaled_dot_product_attention(q, k, v, is_causal=True,
+                                                                 enable_gqa=Hq != Hkv)
+        t_sdpa = timed(run_sdpa, args.steps, args.warmup)
+        sdpa = {"us_per_step": t_sdpa / args.steps * 1e6,
+                "tflops": flops / 2 * args.steps / t_sdpa / 1e12,
+                "note": "torch scaled_dot_product_attention, causal: 4 D flops per pair"}
+    except Exception as exc:  # an SDPA backend may not take this shape
+        sdpa = {"unavailable": str(exc).splitlines()[0][:200]}
+
+    # end to end through the public API: inputs from pinned host memory each step
+    hq, hr, hk, hv = (t.cpu().pin_memory() for t in (q, r, k, v))
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+
+    def run_e2e(k_steps):
+        for _ in range(k_steps):
+            for dst, src in ((q, hq), (r, hr), (k, hk), (v, hv)):
+                dst.copy_(src, non_blocking=True)
+            binding.parallax_prefill(q, r, k, v, out=out, workspace=ws, stream=stream)
+            out_host.copy_(out, non_blocking=True)
+
+    k_e2e = min(args.steps, 20)
+    t_e2e = timed(run_e2e, k_e2e, 2)
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hr, hk, hv))
+    d2h = out_host.numel() * out_host.element_size()
+
+    cpu = None
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        tf, cores, desc, _ = prefill_oracle_sample(shape, min(10.0, args.cpu_seconds))
+        cpu = {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc}
+
+    peak, peak_src = measured_bf16_peak()
+    N = dist.world
+    achieved = flops / kern_s / 1e12
+    clocks = sampler.summary()
+    line = {
+        "metric": PREFILL_METRIC, "value": N * flops * args.steps / t_step / 1e12,
+        "unit": "TFLOP/s", "n_gpus": N, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": t_step / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(cfg, parallelism=f"replicas x{N}" if N > 1 else "single GPU",
+                       l2=("L2 flushed between steps" if flush is not None
+                           else f"inputs ({in_bytes / 1e6:.0f} MB) larger than L2")),
+        "softmax_sdpa": sdpa,
+        "clocks": {k2: clocks[k2] for k2 in ("sm_mhz", "sm_max_mhz", "reasons", "samples")},
+        "e2e": {"value": N * flops * k_e2e / t_e2e / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "us_per_step": t_e2e / k_e2e * 1e6},
+        "gpu_launches": args.steps,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "kernel": "parallax_prefill_kernel", "peak_source": peak_src + " (burst)",
+                     "kernel_us": kern_s * 1e6, "algorithmic_flops_per_launch": flops,
+                     "tensor_flops_issued_per_launch": flops // 8 * 12},
+        "cpu_baseline": cpu,
+    }
+    if dist.rank == 0:
+        print(json.dumps(line))
+    dist.close()
+    return 0
+
+
 # ------------------------------------------------------------- GPU timing ----
 
 def main():
     args = parse_args()
+    if args.prefill:
+        return run_prefill(args)
     if args.impl == "reference":
         return run_reference(args)
 

@@ -186,10 +186,12 @@ int parallax_decode_phase(int phase, int probe, const void* q, const void* r,
  * keys 0..i of kv head h / (Hq/Hkv) (all L keys when causal == 0).
  *  - q, r, out [B][Hq][L][D]; k, v [B][Hkv][L][D]; bf16 inputs (device
  *    pointers, 16-byte aligned); out bf16 or fp32 (out_dtype).
- *  - D is 64 or 128; B and Hq at most 65535.
+ *  - D is 64 or 128; B and Hq at most 65535; scale positive and finite (the
+ *    softmax temperature; PARALLAX_ERR_BAD_SHAPE otherwise).
  *  - The products Q K^T, R K^T, P V and (P o T) V run on the tcgen05 tensor
- *    cores (operands in shared memory, accumulators in tensor memory); the
- *    probabilities enter the value products as bf16 hi + lo pairs.
+ *    cores (accumulators in tensor memory, P read from tensor memory); the
+ *    weights e and e*s enter the value products as exact bf16 hi + lo pairs
+ *    of their values rounded to 17 significant bits.
  *  - workspace: at least 256 bytes, zeroed once; its first word is the device
  *    status word read by parallax_workspace_status.
  * Errors as parallax_decode.

@@ -1,5 +1,5 @@
 // Parallax prefill forward (training shape) on the 5th-generation tensor
-// cores: tcgen05.mma with operands in shared memory and accumulators in TMEM.
+// cores: tcgen05.mma with accumulators in TMEM.
 //
 // parallax-kernel 0.1.0 README, "Training (Triton)": parallax_func(q, r, k, v)
 // maps (B, H, L, D) tensors to (B, H, L, D), causal. Row i of query head h
@@ -8,22 +8,28 @@
 //   l = sum e, b = sum e s, A = sum e v, C = sum e s v,
 //   o_i = A/l + C/l - (b/l)(A/l).
 // Both products are dense contractions here: S = Q K^T and T = R K^T
-// (128 query rows x 64 keys x D) and O_A = P V, O_C = (P o T) V
-// (128 rows x D x 64 keys), so they go through UMMA.
+// (128 query rows x 64 keys x D, operands in shared memory) and O_A = P V,
+// O_C = (P o T) V (128 rows x D x 64 keys, P read from TMEM), so they go
+// through UMMA.
 //
 // One CTA per (128-row query tile, query head, batch row); late (heavier,
-// causal) tiles first. 192 threads:
-//   warp 4  TMA producer: the Q and R tiles once, then 64-key K and V tiles
-//           into a 2-stage ring (128-byte swizzle, the UMMA operand layout)
-//   warp 5  owns the 512 TMEM columns and issues every UMMA (one lane):
-//           S_j, T_j into double-buffered TMEM, then O += P_j V_j
-//   warps 0-3  one query row per thread (= its TMEM lane): causal mask,
-//           online max, e and e*s as bf16 hi + lo pairs written as swizzled
-//           A operands for the PV products, l and b from the same hi + lo
-//           values; O is rescaled in TMEM only when the max grows by more
-//           than 2^8 (otherwise the stale max keeps every e <= 2^8).
-// TMEM columns: S_0 [0,64) T_0 [64,128) S_1 [128,192) T_1 [192,256),
-// O_A [256, 256+D), O_C [256+D, 256+2D).
+// causal) tiles first. 320 threads:
+//   warp 8  TMA producer: the Q and R tiles once, then 64-key K and V tiles
+//           into two 3-stage rings (128-byte swizzle, the UMMA operand layout)
+//   warp 9  owns the 512 TMEM columns and issues every UMMA (one lane), in
+//           the order S_j, T_j, then O += P_{j-1} V_{j-1}: the score products
+//           of a tile run while the softmax of the tile before finishes
+//   warps 0-7  softmax, two threads per query row (TMEM lane): warp w reads
+//           lanes 32 (w % 4).. and keys 32 (w / 4).. of each tile. Each takes
+//           the row max over all 64 keys (no exchange needed) and writes its
+//           32 keys of e and e*s as bf16 hi + lo pairs into the P operand in
+//           TMEM; e and e*s are first rounded to 17 significant bits, so hi +
+//           lo is exact and l, b (summed from the same values) stay consistent
+//           with the weights the products apply. O is rescaled in TMEM only
+//           when the max grows by more than 2^8 (otherwise the stale max keeps
+//           every e <= 2^8); each thread of a row rescales one of O_A, O_C.
+// TMEM columns: S [0,64) T [64,128) P [128,256) (P_hi, P_lo, PT_hi, PT_lo,
+// 32 columns each), O_A [256, 256+D), O_C [256+D, 256+2D).
 // Every wait is bounded; on a timeout the kernel records it, waits (bounded)
 // for its own TMA copies and UMMAs in flight, frees TMEM and returns.
 #pragma once
@@ -35,14 +41,17 @@ namespace plx {
 
 constexpr int kPfRows = 128;     // query rows per CTA (UMMA M)
 constexpr int kPfKeys = 64;      // keys per tile (UMMA N of S, T; K of the PV products)
-constexpr int kPfThreads = 192;  // warps 0-3 softmax, 4 producer, 5 UMMA issuer
+constexpr int kPfSoftmaxWarps = 8;
+constexpr int kPfThreads = 320;  // warps 0-7 softmax, 8 producer, 9 UMMA issuer
+constexpr int kPfStages = 3;     // depth of the K ring and of the V ring
 constexpr int kPfTmemCols = 512;
+constexpr uint32_t kPfColS = 0, kPfColT = 64, kPfColP = 128;
 
 struct PrefillParams {
   void* out;             // [B][Hq][L][D]
   unsigned int* status;  // device status word
   int B, Hq, Hkv, G, L, num_qt, causal;
-  float scale_log2;
+  float scale_log2;      // > 0
   unsigned long long timeout_ns;
 };
 
@@ -51,13 +60,29 @@ struct PfGeom {
   static constexpr int kH = D / 64;
   static constexpr int kQBytes = kH * kPfRows * 128;   // Q (or R) tile
   static constexpr int kKVBytes = kH * kPfKeys * 128;  // K (or V) tile
-  static constexpr int kPBytes = kPfRows * 128;        // one [128 rows][64 keys] bf16 tile
-  static constexpr int kOffQ = 0, kOffR = kQBytes, kOffKV = 2 * kQBytes;
-  static constexpr int kOffP = kOffKV + 2 * 2 * kKVBytes;  // 2 stages of K + V
-  static constexpr int kOffBar = kOffP + 4 * kPBytes;     // P_hi, P_lo, PT_hi, PT_lo
-  static constexpr int kSmem = kOffBar + 128 + 1024;      // barriers, slots, alignment
-  static constexpr int kColOA = 256, kColOC = 256 + D;
+  static constexpr int kOffQ = 0, kOffR = kQBytes, kOffK = 2 * kQBytes;
+  static constexpr int kOffV = kOffK + kPfStages * kKVBytes;
+  static constexpr int kOffRed = kOffV + kPfStages * kKVBytes;  // l, b of both key halves
+  static constexpr int kOffBar = kOffRed + 4 * kPfRows * 4;
+  static constexpr int kSmem = kOffBar + 256 + 1024;            // barriers, slots, alignment
+  static constexpr uint32_t kColOA = 256, kColOC = 256 + D;
 };
+
+// x rounded (half away from zero) to 17 significant bits.
+__device__ __forceinline__ float round17(float x) {
+  return __uint_as_float((__float_as_uint(x) + 0x40u) & 0xFFFFFF80u);
+}
+
+// x0, x1 rounded to 17 significant bits (y), split exactly into bf16 hi + lo:
+// hi = y rounded to nearest bf16, lo = y - hi (at most 8 significant bits, so
+// exact in bf16). Packed as bf16x2 words (x0 in the low half). Returns y0 + y1.
+__device__ __forceinline__ float split_hi_lo(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  const float y0 = round17(x0), y1 = round17(x1);
+  hi = pack_bf16x2(y0, y1);
+  const float l0 = y0 - bf16_lo_to_float(hi), l1 = y1 - bf16_hi_to_float(hi);
+  lo = __byte_perm(__float_as_uint(l0), __float_as_uint(l1), 0x7632);
+  return y0 + y1;
+}
 
 template <int D, bool OUT_F32>
 __global__ void __launch_bounds__(kPfThreads, 1)
@@ -66,7 +91,6 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                             const __grid_constant__ CUtensorMap tmK,
                             const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
   using Geo = PfGeom<D>;
-  constexpr int kH = Geo::kH;
   constexpr uint32_t kIdescS = umma_idesc_bf16(kPfRows, kPfKeys, false);
   constexpr uint32_t kIdescPV = umma_idesc_bf16(kPfRows, D, true);
   const float kNegInf = __int_as_float(0xff800000u);
@@ -75,13 +99,16 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* const gbase = smem_raw + (base - raw);
-  const uint32_t sQ = base + Geo::kOffQ, sR = base + Geo::kOffR, sKV = base + Geo::kOffKV;
-  const uint32_t sP = base + Geo::kOffP;
+  const uint32_t sQ = base + Geo::kOffQ, sR = base + Geo::kOffR;
+  const uint32_t sK = base + Geo::kOffK, sV = base + Geo::kOffV;
   const uint32_t bar = base + Geo::kOffBar;
-  const uint32_t bar_q = bar, bar_kv_full = bar + 8, bar_kv_empty = bar + 24;
-  const uint32_t bar_s = bar + 40, bar_p = bar + 56, bar_o = bar + 64, bar_drain = bar + 72;
-  uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(gbase + Geo::kOffBar + 96);
-  volatile int* const abort_flag = reinterpret_cast<volatile int*>(gbase + Geo::kOffBar + 100);
+  const uint32_t bar_q = bar, k_full = bar + 8, k_empty = bar + 32, v_full = bar + 56,
+                 v_empty = bar + 80;
+  const uint32_t s_full = bar + 104, s_free = bar + 112, p_full = bar + 120, o_done = bar + 128,
+                 bar_drain = bar + 136;
+  uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(gbase + Geo::kOffBar + 144);
+  volatile int* const abort_flag = reinterpret_cast<volatile int*>(gbase + Geo::kOffBar + 148);
+  float* const red = reinterpret_cast<float*>(gbase + Geo::kOffRed);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int qt = p.num_qt - 1 - (int)blockIdx.x;  // heavy causal tiles first
@@ -92,20 +119,23 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 
   if (tid == 0) {
     mbar_init(bar_q, 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(bar_kv_full + 8 * s, 1);
-      mbar_init(bar_kv_empty + 8 * s, 1);
-      mbar_init(bar_s + 8 * s, 1);
+    for (int s = 0; s < kPfStages; ++s) {
+      mbar_init(k_full + 8 * s, 1);
+      mbar_init(k_empty + 8 * s, 1);
+      mbar_init(v_full + 8 * s, 1);
+      mbar_init(v_empty + 8 * s, 1);
     }
-    mbar_init(bar_p, kPfRows);
-    mbar_init(bar_o, 1);
+    mbar_init(s_full, 1);
+    mbar_init(s_free, kPfSoftmaxWarps);
+    mbar_init(p_full, kPfSoftmaxWarps);
+    mbar_init(o_done, 1);
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
     mbar_fence_init();
   }
-  if (warp == 5) tmem_alloc(smem_u32(tmem_slot), kPfTmemCols);
+  if (warp == 9) tmem_alloc(smem_u32(tmem_slot), kPfTmemCols);
   uint64_t policy = 0;
-  if (tid == 4 * 32) {
+  if (tid == 8 * 32) {
     prefetch_tensormap(&tmQ);
     prefetch_tensormap(&tmR);
     prefetch_tensormap(&tmK);
@@ -117,91 +147,108 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ producer --
     if (lane == 0) {
       bool ok = true;
-      uint32_t issued = 0;  // bit s: stage s has a load in flight of tile `last[s]`
-      int last[2] = {0, 0};
+      int last = -1;  // the last tile whose K and V loads were both started
       mbar_arrive_expect_tx(bar_q, 2 * Geo::kQBytes);
       tma_load_4d(sQ, &tmQ, 0, q0, 0, b * p.Hq + h, bar_q, policy);
       tma_load_4d(sR, &tmR, 0, q0, 0, b * p.Hq + h, bar_q, policy);
-      for (int j = 0; j < nkt && ok; ++j) {
-        const int st = j & 1;
-        if (!mbar_wait_bounded(bar_kv_empty + 8 * st, ((j >> 1) & 1) ^ 1, p.timeout_ns,
-                               abort_flag)) {
+      int st = 0;
+      uint32_t ph = 0;
+      for (int j = 0; j < nkt; ++j) {
+        if (!mbar_wait_bounded(k_empty + 8 * st, ph ^ 1, p.timeout_ns, abort_flag)) {
           ok = false;
           break;
         }
-        const uint32_t full = bar_kv_full + 8 * st;
-        const uint32_t sK = sKV + st * 2 * Geo::kKVBytes;
-        mbar_arrive_expect_tx(full, 2 * Geo::kKVBytes);
-        tma_load_4d(sK, &tmK, 0, j * kPfKeys, 0, b * p.Hkv + g, full, policy);
-        tma_load_4d(sK + Geo::kKVBytes, &tmV, 0, j * kPfKeys, 0, b * p.Hkv + g, full, policy);
-        issued |= 1u << st;
-        last[st] = j;
+        mbar_arrive_expect_tx(k_full + 8 * st, Geo::kKVBytes);
+        tma_load_4d(sK + st * Geo::kKVBytes, &tmK, 0, j * kPfKeys, 0, b * p.Hkv + g,
+                    k_full + 8 * st, policy);
+        if (!mbar_wait_bounded(v_empty + 8 * st, ph ^ 1, p.timeout_ns, abort_flag)) {
+          mbar_wait_bounded(k_full + 8 * st, ph, p.timeout_ns, nullptr);  // K_j in flight
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(v_full + 8 * st, Geo::kKVBytes);
+        tma_load_4d(sV + st * Geo::kKVBytes, &tmV, 0, j * kPfKeys, 0, b * p.Hkv + g,
+                    v_full + 8 * st, policy);
+        last = j;
+        if (++st == kPfStages) {
+          st = 0;
+          ph ^= 1;
+        }
       }
       if (!ok) {
         *abort_flag = 1;
         atomicOr(p.status, 1u /* PARALLAX_DEVICE_STATUS_TIMEOUT */);
       }
-      // Wait (bounded) until every copy this CTA started has landed.
+      // Wait (bounded) until every copy this CTA started has landed: the
+      // latest load into each stage is the last one started there.
       mbar_wait_bounded(bar_q, 0, p.timeout_ns, nullptr);
-      for (int s = 0; s < 2; ++s)
-        if (issued & (1u << s))
-          mbar_wait_bounded(bar_kv_full + 8 * s, (last[s] >> 1) & 1, p.timeout_ns, nullptr);
+      for (int j = max(0, last - kPfStages + 1); j <= last; ++j) {
+        const int s = j % kPfStages;
+        const uint32_t par = (uint32_t)(j / kPfStages) & 1u;
+        mbar_wait_bounded(k_full + 8 * s, par, p.timeout_ns, nullptr);
+        mbar_wait_bounded(v_full + 8 * s, par, p.timeout_ns, nullptr);
+      }
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------------- UMMA issuer --
     if (lane == 0) {
       bool ok = mbar_wait_bounded(bar_q, 0, p.timeout_ns, abort_flag);
       tc_fence_after_sync();
       for (int jj = 0; jj <= nkt && ok; ++jj) {
-        if (jj < nkt) {  // S_jj = Q K^T, T_jj = R K^T
-          const int st = jj & 1;
-          if (!mbar_wait_bounded(bar_kv_full + 8 * st, (jj >> 1) & 1, p.timeout_ns, abort_flag)) {
+        if (jj < nkt) {  // S_jj = Q K^T, T_jj = R K^T once the softmax has read S_jj-1
+          const int st = jj % kPfStages;
+          const uint32_t par = (uint32_t)(jj / kPfStages) & 1u;
+          if ((jj > 0 && !mbar_wait_bounded(s_free, (jj - 1) & 1, p.timeout_ns, abort_flag)) ||
+              !mbar_wait_bounded(k_full + 8 * st, par, p.timeout_ns, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after_sync();
-          const uint32_t sK = sKV + st * 2 * Geo::kKVBytes;
-          const uint32_t dS = tmem + 128 * st, dT = dS + 64;
+          const uint32_t sKs = sK + st * Geo::kKVBytes;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t ko = (kk >> 2) * (kPfKeys * 128) + (kk & 3) * 32;
             const uint32_t qo = (kk >> 2) * (kPfRows * 128) + (kk & 3) * 32;
-            umma_bf16(dS, umma_smem_desc(sQ + qo, 16, 1024), umma_smem_desc(sK + ko, 16, 1024),
-                      kIdescS, kk > 0);
+            umma_bf16(tmem + kPfColS, umma_smem_desc(sQ + qo, 16, 1024),
+                      umma_smem_desc(sKs + ko, 16, 1024), kIdescS, kk > 0);
           }
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t ko = (kk >> 2) * (kPfKeys * 128) + (kk & 3) * 32;
             const uint32_t qo = (kk >> 2) * (kPfRows * 128) + (kk & 3) * 32;
-            umma_bf16(dT, umma_smem_desc(sR + qo, 16, 1024), umma_smem_desc(sK + ko, 16, 1024),
-                      kIdescS, kk > 0);
+            umma_bf16(tmem + kPfColT, umma_smem_desc(sR + qo, 16, 1024),
+                      umma_smem_desc(sKs + ko, 16, 1024), kIdescS, kk > 0);
           }
-          umma_commit(bar_s + 8 * st);
+          umma_commit(s_full);
+          umma_commit(k_empty + 8 * st);
         }
         if (jj >= 1) {  // O_A += P V, O_C += (P o T) V for tile j = jj - 1
-          const int j = jj - 1, st = j & 1;
-          if (!mbar_wait_bounded(bar_p, j & 1, p.timeout_ns, abort_flag)) {
+          const int j = jj - 1, st = j % kPfStages;
+          const uint32_t par = (uint32_t)(j / kPfStages) & 1u;
+          if (!mbar_wait_bounded(p_full, j & 1, p.timeout_ns, abort_flag) ||
+              !mbar_wait_bounded(v_full + 8 * st, par, p.timeout_ns, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after_sync();
-          const uint32_t sV = sKV + st * 2 * Geo::kKVBytes + Geo::kKVBytes;
+          const uint32_t sVs = sV + st * Geo::kKVBytes;
 #pragma unroll
           for (int pm = 0; pm < 4; ++pm) {  // P_hi, P_lo -> O_A; PT_hi, PT_lo -> O_C
             const uint32_t dO = tmem + (pm < 2 ? Geo::kColOA : Geo::kColOC);
 #pragma unroll
             for (int kk = 0; kk < kPfKeys / 16; ++kk) {
               const bool acc = !(j == 0 && (pm & 1) == 0 && kk == 0);
-              umma_bf16(dO, umma_smem_desc(sP + pm * Geo::kPBytes + kk * 32, 16, 1024),
-                        umma_smem_desc(sV + kk * 16 * 128, kPfKeys * 128, 1024), kIdescPV, acc);
+              umma_bf16_ts(dO, tmem + kPfColP + 32 * pm + 8 * kk,
+                           umma_smem_desc(sVs + kk * 16 * 128, kPfKeys * 128, 1024), kIdescPV,
+                           acc);
             }
           }
-          umma_commit(bar_o);
-          umma_commit(bar_kv_empty + 8 * st);
+          umma_commit(o_done);
+          umma_commit(v_empty + 8 * st);
         }
       }
       if (!ok) {
@@ -212,49 +259,48 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       mbar_wait_bounded(bar_drain, 0, p.timeout_ns, nullptr);
     }
   } else {
-    // ------------------------------------------- softmax: one row / thread --
-    const int r = tid, qi = q0 + r;
-    const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+    // ------------------------------------- softmax: two threads per row --
+    const int quarter = warp & 3, half = warp >> 2;
+    const int r = quarter * 32 + lane, qi = q0 + r;
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const uint32_t tS = tmem + lane_base + kPfColS, tT = tmem + lane_base + kPfColT;
+    const uint32_t tP = tmem + lane_base + kPfColP + 16 * half;  // this half's 16 columns
+    const float c = p.scale_log2;
     float m_used = kNegInf, l = 0.f, bsum = 0.f;
     bool ok = true;
-    for (int j = 0; j < nkt && ok; ++j) {
-      const int sb = j & 1;
-      if (!mbar_wait_bounded(bar_s + 8 * sb, (j >> 1) & 1, p.timeout_ns, abort_flag)) {
+    for (int j = 0; j < nkt; ++j) {
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(s_full, j & 1, p.timeout_ns, abort_flag))) {
         ok = false;
+        *abort_flag = 1;
         break;
       }
       tc_fence_after_sync();
-      float sv[64], tv[64];
-      {
-        float a[32], c[32];
-        tmem_ld32(tmem + lane_base + 128 * sb, a);
-        tmem_ld32(tmem + lane_base + 128 * sb + 32, c);
-        tmem_wait_ld();
-#pragma unroll
-        for (int x = 0; x < 32; ++x) {
-          sv[x] = a[x];
-          sv[32 + x] = c[x];
-        }
-        tmem_ld32(tmem + lane_base + 128 * sb + 64, a);
-        tmem_ld32(tmem + lane_base + 128 * sb + 96, c);
-        tmem_wait_ld();
-#pragma unroll
-        for (int x = 0; x < 32; ++x) {
-          tv[x] = a[x];
-          tv[32 + x] = c[x];
-        }
-      }
-      // causal mask and the row max of this tile (log2 domain)
-      const int k0 = j * kPfKeys;
-      const int klim = p.causal ? min(kend, qi + 1) : kend;  // keys k0 + x < klim are seen
+      float sv[32], so[32], tv[32];
+      tmem_ld32(tS + 32 * half, sv);
+      tmem_ld32(tS + 32 * (half ^ 1), so);
+      tmem_ld32(tT + 32 * half, tv);
+      tmem_wait_ld();
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_free);
+      // causal mask (only tiles that reach past this tile's first row or the
+      // end of the sequence need one) and the row max over all 64 keys
+      const int k0 = j * kPfKeys, kown = k0 + 32 * half, kother = k0 + 32 * (half ^ 1);
       float mx = kNegInf;
+      if (k0 + kPfKeys <= (p.causal ? min(kend, q0 + 1) : kend)) {
 #pragma unroll
-      for (int x = 0; x < 64; ++x) {
-        const bool valid = k0 + x < klim;
-        sv[x] = valid ? sv[x] * p.scale_log2 : kNegInf;
-        tv[x] = valid ? tv[x] : 0.f;
-        mx = fmaxf(mx, sv[x]);
+        for (int x = 0; x < 32; ++x) mx = fmaxf(mx, fmaxf(sv[x], so[x]));
+      } else {
+        const int klim = p.causal ? min(kend, qi + 1) : kend;  // keys below klim are seen
+#pragma unroll
+        for (int x = 0; x < 32; ++x) {
+          const bool own = kown + x < klim;
+          sv[x] = own ? sv[x] : kNegInf;
+          tv[x] = own ? tv[x] : 0.f;
+          mx = fmaxf(mx, fmaxf(sv[x], kother + x < klim ? so[x] : kNegInf));
+        }
       }
+      mx *= c;  // the scale is positive: this is the max of the scaled scores
       // lazy rescale: keep the stale max unless this tile exceeds it by 2^8
       float alpha = 1.f;
       const bool grow = mx > m_used + 8.f;
@@ -262,73 +308,68 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         alpha = m_used == kNegInf ? 0.f : ex2_approx(m_used - mx);
         m_used = mx;
       }
-      // the previous PV product must be done: P is single-buffered and O may be rescaled
+      const float neg_m = -m_used;
+      // e and e*s of this thread's 32 keys as exact bf16 hi + lo pairs
+      uint32_t ph[16], pl[16], th[16], tl[16];
+      float lt = 0.f, bt = 0.f;
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const float e0 = ex2_approx(fmaf(sv[2 * u], c, neg_m));
+        const float e1 = ex2_approx(fmaf(sv[2 * u + 1], c, neg_m));
+        lt += split_hi_lo(e0, e1, ph[u], pl[u]);
+        // e*s from the rounded e: the weights P applies
+        const float es0 = round17(e0) * tv[2 * u];
+        const float es1 = round17(e1) * tv[2 * u + 1];
+        bt += split_hi_lo(es0, es1, th[u], tl[u]);
+      }
+      // the previous PV products must be done: P is single-buffered and O may be rescaled
       if (j > 0) {
-        if (!mbar_wait_bounded(bar_o, (j - 1) & 1, p.timeout_ns, abort_flag)) {
+        if (!__all_sync(0xffffffffu,
+                        mbar_wait_bounded(o_done, (j - 1) & 1, p.timeout_ns, abort_flag))) {
           ok = false;
+          *abort_flag = 1;
           break;
         }
         tc_fence_after_sync();
         if (grow) {
+          const uint32_t tO = tmem + lane_base + (half ? Geo::kColOC : Geo::kColOA);
 #pragma unroll 1
-          for (int c0 = 0; c0 < 2 * D; c0 += 32) {
+          for (int c0 = 0; c0 < D; c0 += 32) {
             float o[32];
-            tmem_ld32(tmem + lane_base + Geo::kColOA + c0, o);
+            tmem_ld32(tO + c0, o);
             tmem_wait_ld();
 #pragma unroll
             for (int x = 0; x < 32; ++x) o[x] *= alpha;
-            tmem_st32(tmem + lane_base + Geo::kColOA + c0, o);
+            tmem_st32(tO + c0, o);
           }
-          tmem_wait_st();
         }
       }
-      l *= alpha;
-      bsum *= alpha;
-      // e and e*s as bf16 hi + lo, written row r of the four swizzled P tiles
-#pragma unroll
-      for (int c8 = 0; c8 < 8; ++c8) {
-        uint32_t ph[4], pl[4], th[4], tl[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int x = 8 * c8 + 2 * u;
-          const float e0 = ex2_approx(sv[x] - m_used), e1 = ex2_approx(sv[x + 1] - m_used);
-          const float es0 = e0 * tv[x], es1 = e1 * tv[x + 1];
-          ph[u] = pack_bf16x2(e0, e1);
-          pl[u] = pack_bf16x2(e0 - bf16_lo_to_float(ph[u]), e1 - bf16_hi_to_float(ph[u]));
-          th[u] = pack_bf16x2(es0, es1);
-          tl[u] = pack_bf16x2(es0 - bf16_lo_to_float(th[u]), es1 - bf16_hi_to_float(th[u]));
-          l += (bf16_lo_to_float(ph[u]) + bf16_lo_to_float(pl[u])) +
-               (bf16_hi_to_float(ph[u]) + bf16_hi_to_float(pl[u]));
-          bsum += (bf16_lo_to_float(th[u]) + bf16_lo_to_float(tl[u])) +
-                  (bf16_hi_to_float(th[u]) + bf16_hi_to_float(tl[u]));
-        }
-        const uint32_t off = r * 128 + ((c8 ^ (r & 7)) << 4);
-        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(sP + off), "r"(ph[0]),
-                     "r"(ph[1]), "r"(ph[2]), "r"(ph[3])
-                     : "memory");
-        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(sP + Geo::kPBytes + off),
-                     "r"(pl[0]), "r"(pl[1]), "r"(pl[2]), "r"(pl[3])
-                     : "memory");
-        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(sP + 2 * Geo::kPBytes + off),
-                     "r"(th[0]), "r"(th[1]), "r"(th[2]), "r"(th[3])
-                     : "memory");
-        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(sP + 3 * Geo::kPBytes + off),
-                     "r"(tl[0]), "r"(tl[1]), "r"(tl[2]), "r"(tl[3])
-                     : "memory");
-      }
-      fence_proxy_async_smem();  // the tensor cores read P through the async proxy
+      l = l * alpha + lt;
+      bsum = bsum * alpha + bt;
+      tmem_st16(tP + 0 * 32, ph);
+      tmem_st16(tP + 1 * 32, pl);
+      tmem_st16(tP + 2 * 32, th);
+      tmem_st16(tP + 3 * 32, tl);
+      tmem_wait_st();
       tc_fence_before_sync();
-      mbar_arrive(bar_p);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
     }
-    // epilogue: o = A/l + C/l - (b/l)(A/l)
-    if (ok && mbar_wait_bounded(bar_o, (nkt - 1) & 1, p.timeout_ns, abort_flag)) {
+    // epilogue: l and b of the two key halves, then o = A/l + C/l - (b/l)(A/l)
+    red[half * kPfRows + r] = l;
+    red[(2 + half) * kPfRows + r] = bsum;
+    asm volatile("bar.sync 1, %0;" ::"n"(kPfSoftmaxWarps * 32) : "memory");
+    const float lsum = red[r] + red[kPfRows + r];
+    const float bfull = red[2 * kPfRows + r] + red[3 * kPfRows + r];
+    if (ok && __all_sync(0xffffffffu,
+                         mbar_wait_bounded(o_done, (nkt - 1) & 1, p.timeout_ns, abort_flag))) {
       tc_fence_after_sync();
-      const float inv = 1.f / l, bl = bsum * inv;
+      const float inv = 1.f / lsum, bl = bfull * inv;
 #pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        float a[32], c[32];
+      for (int c0 = half * (D / 2); c0 < (half + 1) * (D / 2); c0 += 32) {
+        float a[32], cc[32];
         tmem_ld32(tmem + lane_base + Geo::kColOA + c0, a);
-        tmem_ld32(tmem + lane_base + Geo::kColOC + c0, c);
+        tmem_ld32(tmem + lane_base + Geo::kColOC + c0, cc);
         tmem_wait_ld();
         if (qi < p.L) {
           const size_t oi = (((size_t)b * p.Hq + h) * p.L + qi) * D + c0;
@@ -338,7 +379,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 #pragma unroll
             for (int y = 0; y < 4; ++y) {
               const float vbar = a[x + y] * inv;
-              o4[y] = vbar + c[x + y] * inv - bl * vbar;
+              o4[y] = vbar + cc[x + y] * inv - bl * vbar;
             }
             if (OUT_F32) {
               *reinterpret_cast<float4*>(static_cast<float*>(p.out) + oi + x) =
@@ -352,7 +393,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           }
         }
       }
-    } else if (ok) {
+    } else {
       ok = false;
     }
     if (!ok) {
@@ -364,7 +405,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
-  if (warp == 5) tmem_dealloc(tmem, kPfTmemCols);
+  if (warp == 9) tmem_dealloc(tmem, kPfTmemCols);
 }
 
 }  // namespace plx

@@ -473,6 +473,7 @@ extern "C" int parallax_prefill(const void* q, const void* r, const void* k, con
   if (!q || !r || !k || !v || !out || !workspace) return PARALLAX_ERR_NULL_POINTER;
   if (B < 1 || Hq < 1 || Hkv < 1 || L < 1 || Hq % Hkv != 0 || B > 65535 || Hq > 65535)
     return PARALLAX_ERR_BAD_SHAPE;
+  if (!(scale > 0.f) || !(scale < 3.0e38f)) return PARALLAX_ERR_BAD_SHAPE;  // positive, finite
   if (D != 64 && D != 128) return PARALLAX_ERR_UNSUPPORTED_HEAD_DIM;
   if (out_dtype != PARALLAX_DTYPE_BF16 && out_dtype != PARALLAX_DTYPE_F32)
     return PARALLAX_ERR_UNSUPPORTED_DTYPE;

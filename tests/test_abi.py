@@ -127,3 +127,27 @@ def test_phase_selector(lib):
     rc = lib.parallax_decode_phase(3, 1, 16, 16, 16, 16, 16, 16, 1, 16, 8, 128,
                                    ctypes.c_float(0.1), None, 64, 0, 0, 4, 16, 1 << 20)
     assert rc == -10
+
+
+def test_prefill_argument_errors_before_launch(lib):
+    fn = lib.parallax_prefill
+    fn.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_int] * 5 + [ctypes.c_float, ctypes.c_int,
+                                                                ctypes.c_void_p, ctypes.c_int,
+                                                                ctypes.c_void_p, ctypes.c_size_t]
+    fn.restype = ctypes.c_int
+
+    def call(q=16, out=16, B=1, Hq=4, Hkv=2, L=64, D=128, scale=0.1, outd=0, ws=16, wsb=256):
+        return fn(q, 16, 16, 16, out, B, Hq, Hkv, L, D, scale, 1, None, outd, ws, wsb)
+
+    assert call(q=None) == ENULL
+    assert call(ws=None) == ENULL
+    assert call(Hq=3) == ESHAPE
+    assert call(L=0) == ESHAPE
+    assert call(scale=0.0) == ESHAPE  # the softmax temperature must be positive
+    assert call(scale=-0.1) == ESHAPE
+    assert call(scale=float("inf")) == ESHAPE
+    assert call(scale=float("nan")) == ESHAPE
+    assert call(D=96) == EHEAD
+    assert call(outd=2) == EDTYPE
+    assert call(out=8) == EALIGN
+    assert call(wsb=100) == EWS
