@@ -202,6 +202,33 @@ int parallax_prefill(const void* q, const void* r, const void* k, const void* v,
                      size_t workspace_bytes);
 
 /*
+ * The packed variable-length forward: parallax-kernel 0.1.0 README, "Helion
+ * kernels (experimental)" and "Install" name parallax_varlen_func beside
+ * parallax_func ("training (dense + varlen)"). The pages give no signature; this
+ * takes the usual packed form: sequence b occupies rows cu_seqlens[b] ..
+ * cu_seqlens[b+1]-1 of the token dimension and each row attends (causally,
+ * unless causal == 0) to the keys of its own sequence only, with the
+ * arithmetic of parallax_prefill.
+ *  - q, r, out [total_tokens][Hq][D]; k, v [total_tokens][Hkv][D]; bf16 inputs
+ *    (device pointers, 16-byte aligned); out bf16 or fp32 (out_dtype).
+ *  - cu_seqlens: device int32 [B + 1], non-decreasing, cu_seqlens[0] = 0,
+ *    cu_seqlens[B] = total_tokens. Values outside [0, total_tokens] or a
+ *    decreasing pair are clamped on the device (no row outside the buffers is
+ *    touched) and set PARALLAX_DEVICE_STATUS_SEQLEN_CLAMPED.
+ *  - max_seqlen: the longest sequence (it sizes the grid; a longer sequence
+ *    sets PARALLAX_DEVICE_STATUS_SEQLEN_CLAMPED and its first rows are not
+ *    written). 1 <= max_seqlen <= total_tokens.
+ *  - Rows of a neighbouring sequence may be read into a tile and masked out
+ *    (weight 0), so inputs must be finite.
+ *  - workspace and errors as parallax_prefill.
+ */
+int parallax_varlen_prefill(const void* q, const void* r, const void* k, const void* v,
+                            const int32_t* cu_seqlens, void* out, int B, int total_tokens,
+                            int max_seqlen, int Hq, int Hkv, int D, float scale, int causal,
+                            void* stream, int out_dtype, void* workspace,
+                            size_t workspace_bytes);
+
+/*
  * Synchronise the current device, then read (and, if clear != 0, zero) the
  * device status word at the start of a workspace. *device_status receives PARALLAX_DEVICE_STATUS_* bits;
  * the return value maps them to a status: PARALLAX_ERR_DEVICE_TIMEOUT if a

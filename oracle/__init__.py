@@ -124,6 +124,29 @@ class Oracle:
         self._check(rc, "oracle_parallax_prefill")
         return out
 
+    def parallax_varlen_prefill(self, q, r, k, v, cu_seqlens, scale, causal=True):
+        """Packed variable-length forward: q, r [total, Hq, D], k, v [total,
+        Hkv, D]; sequence b is rows cu_seqlens[b]:cu_seqlens[b+1] and attends to
+        its own keys only. Each sequence goes through parallax_prefill on its
+        own, moved to the [1, H, len, D] layout and back."""
+        q, r, k, v = _f64(q), _f64(r), _f64(k), _f64(v)
+        if hasattr(cu_seqlens, "detach"):
+            cu_seqlens = cu_seqlens.detach().cpu().numpy()
+        cu = np.asarray(cu_seqlens, dtype=np.int64)
+        if q.ndim != 3 or r.shape != q.shape or k.ndim != 3 or v.shape != k.shape:
+            raise ValueError("expected q, r [total,Hq,D] and k, v [total,Hkv,D]")
+        if cu.ndim != 1 or cu[0] != 0 or cu[-1] != q.shape[0] or np.any(np.diff(cu) < 0):
+            raise ValueError("cu_seqlens must rise from 0 to total")
+        out = np.zeros_like(q)
+        for b in range(len(cu) - 1):
+            a, e = int(cu[b]), int(cu[b + 1])
+            if e == a:
+                continue
+            seq = [np.ascontiguousarray(x[a:e].transpose(1, 0, 2))[None] for x in (q, r, k, v)]
+            o = self.parallax_prefill(*seq, scale, causal)
+            out[a:e] = o[0].transpose(1, 0, 2)
+        return out
+
     # The default used by parity checks: the definition (covariance) form.
     def parallax_decode(self, q, r, k, v, seqlens, scale):
         return self.parallax_covariance(q, r, k, v, seqlens, scale)
@@ -164,6 +187,10 @@ def parallax_decode(*a, **kw):
 
 def parallax_prefill(*a, **kw):
     return default().parallax_prefill(*a, **kw)
+
+
+def parallax_varlen_prefill(*a, **kw):
+    return default().parallax_varlen_prefill(*a, **kw)
 
 
 def num_threads() -> int:

@@ -66,6 +66,43 @@ def _check(status: int, what: str) -> None:
         raise RuntimeError(f"{what} failed: {parallax_status_string(status)} (status {status})")
 
 
+def parallax_varlen_prefill(q, r, k, v, cu_seqlens, max_seqlen: Optional[int] = None,
+                            scale: Optional[float] = None, causal: bool = True, out=None,
+                            out_dtype=None, workspace=None, stream=None):
+    """Packed variable-length forward (the README's parallax_varlen_func):
+    q, r [total, Hq, D], k, v [total, Hkv, D] bf16, cu_seqlens int32 [B + 1] on
+    the device; sequence b is rows cu_seqlens[b]:cu_seqlens[b+1]."""
+    lib = load_library()
+    fn = lib.parallax_varlen_prefill
+    vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    fn.argtypes = [vp] * 6 + [i] * 6 + [f, i, vp, i, vp, ctypes.c_size_t]
+    fn.restype = i
+    for name, t in (("q", q), ("r", r), ("k", k), ("v", v)):
+        if not t.is_cuda or not t.is_contiguous() or t.dtype != torch.bfloat16 or t.dim() != 3:
+            raise ValueError(f"{name} must be a contiguous 3-D bf16 CUDA tensor")
+    total, Hq, D = q.shape
+    if r.shape != q.shape or k.shape != v.shape or k.shape[0] != total or k.shape[2] != D:
+        raise ValueError("expected q, r [total, Hq, D] and k, v [total, Hkv, D]")
+    if (not cu_seqlens.is_cuda or cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1
+            or not cu_seqlens.is_contiguous()):
+        raise ValueError("cu_seqlens must be a contiguous 1-D int32 CUDA tensor")
+    B = cu_seqlens.numel() - 1
+    if max_seqlen is None:  # one device read; pass it to stay asynchronous
+        max_seqlen = int((cu_seqlens[1:] - cu_seqlens[:-1]).max().item()) if B > 0 else 0
+    if out is None:
+        out = torch.empty_like(q, dtype=out_dtype if out_dtype is not None else q.dtype)
+    if workspace is None:
+        workspace = torch.zeros(256, dtype=torch.uint8, device=q.device)
+    buf = workspace.buffer if isinstance(workspace, Workspace) else workspace
+    scale = D ** -0.5 if scale is None else scale
+    rc = fn(q.data_ptr(), r.data_ptr(), k.data_ptr(), v.data_ptr(), cu_seqlens.data_ptr(),
+            out.data_ptr(), B, total, int(max_seqlen), Hq, k.shape[1], D, float(scale),
+            int(bool(causal)), _stream(stream), _DTYPE_CODE[out.dtype], buf.data_ptr(),
+            buf.numel())
+    _check(rc, "parallax_varlen_prefill")
+    return out
+
+
 def parallax_choose_splits(B: int, Hkv: int, Lmax: int, sm_count: int = 0) -> int:
     n = load_library().parallax_choose_splits(B, Hkv, Lmax, sm_count)
     if n < 0:

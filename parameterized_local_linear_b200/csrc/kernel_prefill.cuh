@@ -48,10 +48,12 @@ constexpr int kPfTmemCols = 512;
 constexpr uint32_t kPfColS = 0, kPfColT = 64, kPfColP = 128;
 
 struct PrefillParams {
-  void* out;             // [B][Hq][L][D]
-  unsigned int* status;  // device status word
+  void* out;                // dense [B][Hq][L][D]; packed [total][Hq][D]
+  unsigned int* status;     // device status word
+  const int* cu_seqlens;    // packed layout: [B + 1] sequence starts (nullptr when dense)
   int B, Hq, Hkv, G, L, num_qt, causal;
-  float scale_log2;      // > 0
+  int total;                // packed layout: rows of q, k (cu_seqlens is clamped to it)
+  float scale_log2;         // > 0
   unsigned long long timeout_ns;
 };
 
@@ -84,7 +86,10 @@ __device__ __forceinline__ float split_hi_lo(float x0, float x1, uint32_t& hi, u
   return y0 + y1;
 }
 
-template <int D, bool OUT_F32>
+// VARLEN: the packed layout of parallax_varlen_func (q, r, out [total][Hq][D],
+// k, v [total][Hkv][D], sequence b in rows cu_seqlens[b] .. cu_seqlens[b+1]);
+// otherwise the dense [B][H][L][D] layout.
+template <int D, bool OUT_F32, bool VARLEN>
 __global__ void __launch_bounds__(kPfThreads, 1)
     parallax_prefill_kernel(const __grid_constant__ CUtensorMap tmQ,
                             const __grid_constant__ CUtensorMap tmR,
@@ -111,11 +116,26 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   float* const red = reinterpret_cast<float*>(gbase + Geo::kOffRed);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int qt = p.num_qt - 1 - (int)blockIdx.x;  // heavy causal tiles first
   const int h = blockIdx.y, b = blockIdx.z, g = h / p.G;
+  // this sequence: its length L and, packed, its first row s0
+  int L = p.L, s0 = 0;
+  if (VARLEN) {
+    const int a = __ldg(p.cu_seqlens + b), e = __ldg(p.cu_seqlens + b + 1);
+    s0 = min(max(a, 0), p.total);
+    L = min(max(e, s0), p.total) - s0;
+    const bool bad = s0 != a || s0 + L != e;  // outside [0, total] or decreasing
+    if (tid == 0 && blockIdx.x == 0 && h == 0 && (bad || (L + kPfRows - 1) / kPfRows > (int)gridDim.x))
+      atomicOr(p.status, 2u /* PARALLAX_DEVICE_STATUS_SEQLEN_CLAMPED */);
+  }
+  const int num_qt = VARLEN ? (L + kPfRows - 1) / kPfRows : p.num_qt;
+  if ((int)blockIdx.x >= num_qt) return;  // shorter sequence: nothing for this CTA
+  const int qt = num_qt - 1 - (int)blockIdx.x;  // heavy causal tiles first
   const int q0 = qt * kPfRows;
-  const int kend = p.causal ? min(p.L, q0 + kPfRows) : p.L;  // keys this tile can see
+  const int kend = p.causal ? min(L, q0 + kPfRows) : L;  // keys this tile can see
   const int nkt = (kend + kPfKeys - 1) / kPfKeys;
+  // TMA coordinates: (row, item) of the Q, R box and of the K, V boxes
+  const int qrow = VARLEN ? s0 + q0 : q0, qitem = VARLEN ? h : b * p.Hq + h;
+  const int krow = VARLEN ? s0 : 0, kitem = VARLEN ? g : b * p.Hkv + g;
 
   if (tid == 0) {
     mbar_init(bar_q, 1);
@@ -153,8 +173,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       bool ok = true;
       int last = -1;  // the last tile whose K and V loads were both started
       mbar_arrive_expect_tx(bar_q, 2 * Geo::kQBytes);
-      tma_load_4d(sQ, &tmQ, 0, q0, 0, b * p.Hq + h, bar_q, policy);
-      tma_load_4d(sR, &tmR, 0, q0, 0, b * p.Hq + h, bar_q, policy);
+      tma_load_4d(sQ, &tmQ, 0, qrow, 0, qitem, bar_q, policy);
+      tma_load_4d(sR, &tmR, 0, qrow, 0, qitem, bar_q, policy);
       int st = 0;
       uint32_t ph = 0;
       for (int j = 0; j < nkt; ++j) {
@@ -163,7 +183,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           break;
         }
         mbar_arrive_expect_tx(k_full + 8 * st, Geo::kKVBytes);
-        tma_load_4d(sK + st * Geo::kKVBytes, &tmK, 0, j * kPfKeys, 0, b * p.Hkv + g,
+        tma_load_4d(sK + st * Geo::kKVBytes, &tmK, 0, krow + j * kPfKeys, 0, kitem,
                     k_full + 8 * st, policy);
         if (!mbar_wait_bounded(v_empty + 8 * st, ph ^ 1, p.timeout_ns, abort_flag)) {
           mbar_wait_bounded(k_full + 8 * st, ph, p.timeout_ns, nullptr);  // K_j in flight
@@ -171,7 +191,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           break;
         }
         mbar_arrive_expect_tx(v_full + 8 * st, Geo::kKVBytes);
-        tma_load_4d(sV + st * Geo::kKVBytes, &tmV, 0, j * kPfKeys, 0, b * p.Hkv + g,
+        tma_load_4d(sV + st * Geo::kKVBytes, &tmV, 0, krow + j * kPfKeys, 0, kitem,
                     v_full + 8 * st, policy);
         last = j;
         if (++st == kPfStages) {
@@ -371,8 +391,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         tmem_ld32(tmem + lane_base + Geo::kColOA + c0, a);
         tmem_ld32(tmem + lane_base + Geo::kColOC + c0, cc);
         tmem_wait_ld();
-        if (qi < p.L) {
-          const size_t oi = (((size_t)b * p.Hq + h) * p.L + qi) * D + c0;
+        if (qi < L) {
+          const size_t oi = (VARLEN ? ((size_t)(s0 + qi) * p.Hq + h)
+                                    : (((size_t)b * p.Hq + h) * L + qi)) * D + c0;
 #pragma unroll
           for (int x = 0; x < 32; x += 4) {
             float o4[4];

@@ -442,21 +442,41 @@ int encode_rows_map(CUtensorMap* map, const void* base, int D, int L, long long 
   return r == CUDA_SUCCESS ? PARALLAX_OK : PARALLAX_ERR_CUDA;
 }
 
-template <int D, bool OUT_F32>
+// Packed [total][H][D] bf16 viewed as {64 dims, total rows, D/64 halves, H
+// heads}: a box of `box_rows` consecutive rows of one head lands in the same
+// swizzled layout as encode_rows_map's.
+int encode_packed_map(CUtensorMap* map, const void* base, int D, int total, int H,
+                      int box_rows) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return PARALLAX_ERR_CUDA;
+  cuuint64_t dims[4] = {64, (cuuint64_t)total, (cuuint64_t)(D / 64), (cuuint64_t)H};
+  cuuint64_t strides[3] = {(cuuint64_t)H * D * 2, 128, (cuuint64_t)D * 2};
+  cuuint32_t box[4] = {64, (cuuint32_t)box_rows, (cuuint32_t)(D / 64), 1};
+  cuuint32_t elem[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
+                   strides, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? PARALLAX_OK : PARALLAX_ERR_CUDA;
+}
+
+template <int D, bool OUT_F32, bool VARLEN>
 int launch_prefill(const void* q, const void* r, const void* k, const void* v,
-                   const PrefillParams& prm, int Hq, int Hkv, int L, int B,
-                   cudaStream_t stream) {
-  auto kernel = parallax_prefill_kernel<D, OUT_F32>;
+                   const PrefillParams& prm, int grid_x, cudaStream_t stream) {
+  auto kernel = parallax_prefill_kernel<D, OUT_F32, VARLEN>;
   static int done[256] = {0};
   int st = set_smem_once(kernel, PfGeom<D>::kSmem, done);
   if (st != PARALLAX_OK) return st;
   CUtensorMap tq, tr, tk, tv;
-  if ((st = encode_rows_map(&tq, q, D, L, (long long)B * Hq, kPfRows)) != PARALLAX_OK) return st;
-  if ((st = encode_rows_map(&tr, r, D, L, (long long)B * Hq, kPfRows)) != PARALLAX_OK) return st;
-  if ((st = encode_rows_map(&tk, k, D, L, (long long)B * Hkv, kPfKeys)) != PARALLAX_OK) return st;
-  if ((st = encode_rows_map(&tv, v, D, L, (long long)B * Hkv, kPfKeys)) != PARALLAX_OK) return st;
+  const void* src[4] = {q, r, k, v};
+  CUtensorMap* maps[4] = {&tq, &tr, &tk, &tv};
+  for (int i = 0; i < 4; ++i) {
+    const int H = i < 2 ? prm.Hq : prm.Hkv, rows = i < 2 ? kPfRows : kPfKeys;
+    st = VARLEN ? encode_packed_map(maps[i], src[i], D, prm.total, H, rows)
+                : encode_rows_map(maps[i], src[i], D, prm.L, (long long)prm.B * H, rows);
+    if (st != PARALLAX_OK) return st;
+  }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)prm.num_qt, (unsigned)Hq, (unsigned)B);
+  cfg.gridDim = dim3((unsigned)grid_x, (unsigned)prm.Hq, (unsigned)prm.B);
   cfg.blockDim = dim3(kPfThreads);
   cfg.dynamicSmemBytes = PfGeom<D>::kSmem;
   cfg.stream = stream;
@@ -464,15 +484,22 @@ int launch_prefill(const void* q, const void* r, const void* k, const void* v,
                                                                               : PARALLAX_ERR_CUDA;
 }
 
-}  // namespace
+template <bool VARLEN>
+int dispatch_prefill(const void* q, const void* r, const void* k, const void* v,
+                     const PrefillParams& prm, int D, bool f32, int grid_x, cudaStream_t s) {
+  if (D == 128)
+    return f32 ? launch_prefill<128, true, VARLEN>(q, r, k, v, prm, grid_x, s)
+               : launch_prefill<128, false, VARLEN>(q, r, k, v, prm, grid_x, s);
+  return f32 ? launch_prefill<64, true, VARLEN>(q, r, k, v, prm, grid_x, s)
+             : launch_prefill<64, false, VARLEN>(q, r, k, v, prm, grid_x, s);
+}
 
-extern "C" int parallax_prefill(const void* q, const void* r, const void* k, const void* v,
-                                void* out, int B, int Hq, int Hkv, int L, int D, float scale,
-                                int causal, void* stream, int out_dtype, void* workspace,
-                                size_t workspace_bytes) {
+// The checks both prefill layouts share.
+int check_prefill_args(const void* q, const void* r, const void* k, const void* v, void* out,
+                       int Hq, int Hkv, int D, float scale, int out_dtype, void* workspace,
+                       size_t workspace_bytes) {
   if (!q || !r || !k || !v || !out || !workspace) return PARALLAX_ERR_NULL_POINTER;
-  if (B < 1 || Hq < 1 || Hkv < 1 || L < 1 || Hq % Hkv != 0 || B > 65535 || Hq > 65535)
-    return PARALLAX_ERR_BAD_SHAPE;
+  if (Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || Hq > 65535) return PARALLAX_ERR_BAD_SHAPE;
   if (!(scale > 0.f) || !(scale < 3.0e38f)) return PARALLAX_ERR_BAD_SHAPE;  // positive, finite
   if (D != 64 && D != 128) return PARALLAX_ERR_UNSUPPORTED_HEAD_DIM;
   if (out_dtype != PARALLAX_DTYPE_BF16 && out_dtype != PARALLAX_DTYPE_F32)
@@ -481,6 +508,19 @@ extern "C" int parallax_prefill(const void* q, const void* r, const void* k, con
       !aligned16(workspace))
     return PARALLAX_ERR_MISALIGNED;
   if (workspace_bytes < kWorkspaceHeaderBytes) return PARALLAX_ERR_WORKSPACE_TOO_SMALL;
+  return PARALLAX_OK;
+}
+
+}  // namespace
+
+extern "C" int parallax_prefill(const void* q, const void* r, const void* k, const void* v,
+                                void* out, int B, int Hq, int Hkv, int L, int D, float scale,
+                                int causal, void* stream, int out_dtype, void* workspace,
+                                size_t workspace_bytes) {
+  int st = check_prefill_args(q, r, k, v, out, Hq, Hkv, D, scale, out_dtype, workspace,
+                              workspace_bytes);
+  if (st != PARALLAX_OK) return st;
+  if (B < 1 || L < 1 || B > 65535) return PARALLAX_ERR_BAD_SHAPE;
   PrefillParams prm{};
   prm.out = out;
   prm.status = static_cast<unsigned int*>(workspace);
@@ -493,13 +533,37 @@ extern "C" int parallax_prefill(const void* q, const void* r, const void* k, con
   prm.causal = causal != 0;
   prm.scale_log2 = (float)((double)scale * 1.4426950408889634);
   prm.timeout_ns = kDefaultTimeoutNs;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const bool f32 = out_dtype == PARALLAX_DTYPE_F32;
-  if (D == 128)
-    return f32 ? launch_prefill<128, true>(q, r, k, v, prm, Hq, Hkv, L, B, s)
-               : launch_prefill<128, false>(q, r, k, v, prm, Hq, Hkv, L, B, s);
-  return f32 ? launch_prefill<64, true>(q, r, k, v, prm, Hq, Hkv, L, B, s)
-             : launch_prefill<64, false>(q, r, k, v, prm, Hq, Hkv, L, B, s);
+  return dispatch_prefill<false>(q, r, k, v, prm, D, out_dtype == PARALLAX_DTYPE_F32,
+                                 prm.num_qt, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int parallax_varlen_prefill(const void* q, const void* r, const void* k,
+                                       const void* v, const int32_t* cu_seqlens, void* out,
+                                       int B, int total_tokens, int max_seqlen, int Hq, int Hkv,
+                                       int D, float scale, int causal, void* stream,
+                                       int out_dtype, void* workspace, size_t workspace_bytes) {
+  int st = check_prefill_args(q, r, k, v, out, Hq, Hkv, D, scale, out_dtype, workspace,
+                              workspace_bytes);
+  if (st != PARALLAX_OK) return st;
+  if (!cu_seqlens) return PARALLAX_ERR_NULL_POINTER;
+  if (B < 1 || B > 65535 || total_tokens < 1 || max_seqlen < 1 || max_seqlen > total_tokens)
+    return PARALLAX_ERR_BAD_SHAPE;
+  PrefillParams prm{};
+  prm.out = out;
+  prm.status = static_cast<unsigned int*>(workspace);
+  prm.cu_seqlens = cu_seqlens;
+  prm.B = B;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.G = Hq / Hkv;
+  prm.L = 0;
+  prm.total = total_tokens;
+  prm.causal = causal != 0;
+  prm.scale_log2 = (float)((double)scale * 1.4426950408889634);
+  prm.timeout_ns = kDefaultTimeoutNs;
+  return dispatch_prefill<true>(q, r, k, v, prm, D, out_dtype == PARALLAX_DTYPE_F32,
+                                (max_seqlen + kPfRows - 1) / kPfRows,
+                                static_cast<cudaStream_t>(stream));
 }
 
 extern "C" int parallax_testing_decode_stalled(const void* q, const void* r, const void* k_cache,

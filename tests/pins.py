@@ -344,10 +344,76 @@ def pin_prefill_gqa_mapping(orc):
     close(o, want, 1e-12, "prefill GQA mapping")
 
 
+# ------------------------------------------------------------------- varlen --
+
+def rand_packed(seed, lens=(5, 0, 9, 1, 7), Hq=4, Hkv=2, D=8, r_scale=0.5):
+    rng = np.random.default_rng(seed)
+    total = int(sum(lens))
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    q = rng.standard_normal((total, Hq, D))
+    r = rng.standard_normal((total, Hq, D)) * r_scale
+    k = rng.standard_normal((total, Hkv, D))
+    v = rng.standard_normal((total, Hkv, D))
+    return q, r, k, v, cu
+
+
+def pin_varlen_r_zero_is_masked_sdpa(orc):
+    """r = 0: torch's SDPA over the whole packed token axis with an explicit
+    block-diagonal (and causal) boolean mask, computed independently of the
+    per-sequence split."""
+    q, r, k, v, cu = rand_packed(30)
+    total = q.shape[0]
+    seg = np.repeat(np.arange(len(cu) - 1), np.diff(cu))
+    pos = np.arange(total)
+    for causal in (True, False):
+        mask = seg[:, None] == seg[None, :]
+        if causal:
+            mask &= pos[None, :] <= pos[:, None]
+        qt, kt, vt = (torch.from_numpy(x.transpose(1, 0, 2).copy()) for x in (q, k, v))
+        kt = torch.repeat_interleave(kt, 2, dim=0)
+        vt = torch.repeat_interleave(vt, 2, dim=0)
+        want = torch.nn.functional.scaled_dot_product_attention(
+            qt, kt, vt, attn_mask=torch.from_numpy(mask), scale=0.4).numpy().transpose(1, 0, 2)
+        got = orc.parallax_varlen_prefill(q, np.zeros_like(r), k, v, cu, 0.4, causal)
+        close(got, want, 1e-12, f"varlen r=0 causal={causal}")
+
+
+def pin_varlen_equal_lengths_match_dense(orc):
+    """Equal-length sequences packed along the token axis give the dense
+    [B, H, L, D] forward, row for row."""
+    q, r, k, v = rand_prefill(31, B=3, Hq=4, Hkv=2, L=6, D=8)
+    dense = orc.parallax_prefill(q, r, k, v, 0.3)
+    pack = lambda x: np.ascontiguousarray(x.transpose(0, 2, 1, 3).reshape(-1, x.shape[1], x.shape[3]))
+    cu = np.array([0, 6, 12, 18], dtype=np.int32)
+    got = orc.parallax_varlen_prefill(pack(q), pack(r), pack(k), pack(v), cu, 0.3)
+    close(got, pack(dense), 1e-12, "varlen = dense for equal lengths")
+
+
+def pin_varlen_sequences_isolated(orc):
+    """No row sees another sequence: replacing every token of one sequence
+    (values by NaN) leaves the others' outputs bit-identical."""
+    q, r, k, v, cu = rand_packed(32)
+    o = orc.parallax_varlen_prefill(q, r, k, v, cu, 0.3)
+    a, e = int(cu[2]), int(cu[3])  # the third sequence (9 tokens)
+    q2, r2, k2, v2 = (x.copy() for x in (q, r, k, v))
+    for x in (q2, r2, k2):
+        x[a:e] += 3.0
+    v2[a:e] = np.nan
+    o2 = orc.parallax_varlen_prefill(q2, r2, k2, v2, cu, 0.3)
+    keep = np.ones(q.shape[0], bool)
+    keep[a:e] = False
+    assert np.array_equal(o2[keep], o[keep]), "varlen sequences interact"
+    # row 0 of every non-empty sequence is its own v_0
+    for b in range(len(cu) - 1):
+        if cu[b + 1] > cu[b]:
+            close(o[cu[b]], np.repeat(v[cu[b]], 2, axis=0), 1e-12, "varlen first row")
+
+
 PINS = [pin_hand_examples, pin_r_zero_is_softmax, pin_single_key_returns_v,
         pin_constant_values, pin_value_shift_and_scale, pin_key_translation,
         pin_linear_in_r, pin_key_permutation, pin_forms_agree,
         pin_local_linear_intercept, pin_gqa_mapping, pin_lengths_exact,
         pin_empty_sequence_is_zero, pin_prefill_r_zero_is_sdpa,
         pin_prefill_first_row_and_causality, pin_prefill_local_linear_intercept,
-        pin_prefill_gqa_mapping]
+        pin_prefill_gqa_mapping, pin_varlen_r_zero_is_masked_sdpa,
+        pin_varlen_equal_lengths_match_dense, pin_varlen_sequences_isolated]

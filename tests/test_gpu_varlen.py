@@ -1,0 +1,92 @@
+"""GPU parity of the packed variable-length forward (the README's
+parallax_varlen_func, "Training (dense + varlen)") against the fp64 oracle:
+ragged sequences that span several 128-row query tiles and partial 64-key
+tiles, an empty sequence, GQA, both head dimensions, causal and not, bf16 and
+fp32 outputs, plus the device-side clamping of malformed cu_seqlens."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parameterized_local_linear_b200 import binding
+
+pytestmark = pytest.mark.gpu
+
+TOL = {torch.bfloat16: 2e-2, torch.float32: 1e-4}
+
+
+def make(lens, Hq, Hkv, D, seed, r_scale=0.5):
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    total = int(sum(lens))
+    rnd = lambda H, s=1.0: (torch.randn(total, H, D, device="cuda", generator=g) * s).to(torch.bfloat16)
+    q, r, k, v = rnd(Hq), rnd(Hq, r_scale), rnd(Hkv), rnd(Hkv)
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32, device="cuda")
+    return q, r, k, v, cu
+
+
+def status_bits(ws):
+    """The device status word (first 4 bytes of the workspace), then cleared."""
+    torch.cuda.synchronize()
+    bits = int(ws[:4].view(torch.int32).item())
+    ws.zero_()
+    return bits
+
+
+def scaled_error(got, ref):
+    g = got.float().cpu().double().numpy()
+    assert np.all(np.isfinite(g)), "non-finite output"
+    return float(np.max(np.abs(g - ref) / np.maximum(1.0, np.abs(ref))))
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("Hq,Hkv", [(2, 2), (4, 2)])
+def test_varlen_matches_oracle(D, Hq, Hkv):
+    lens = [1, 130, 64, 0, 257, 5, 128]
+    q, r, k, v, cu = make(lens, Hq, Hkv, D, seed=400 + D + Hq)
+    scale = D ** -0.5
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    for causal in (True, False):
+        want = oracle.parallax_varlen_prefill(q, r, k, v, cu, scale, causal)
+        for out_dtype in (torch.bfloat16, torch.float32):
+            got = binding.parallax_varlen_prefill(q, r, k, v, cu, max(lens), scale=scale,
+                                                  causal=causal, out_dtype=out_dtype, workspace=ws)
+            err = scaled_error(got, want)
+            assert err <= TOL[out_dtype], (D, Hq, Hkv, causal, out_dtype, err)
+    torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32).item()) == 0
+
+
+def test_varlen_equal_lengths_match_dense_kernel():
+    B, Hq, Hkv, L, D = 3, 4, 2, 200, 128
+    g = torch.Generator(device="cuda").manual_seed(410)
+    mk = lambda H: torch.randn(B, H, L, D, device="cuda", generator=g).to(torch.bfloat16)
+    q, r, k, v = mk(Hq), mk(Hq), mk(Hkv), mk(Hkv)
+    dense = binding.parallax_prefill(q, r, k, v, out_dtype=torch.float32)
+    pack = lambda x: x.transpose(1, 2).reshape(B * L, x.shape[1], D).contiguous()
+    cu = torch.arange(0, B * L + 1, L, dtype=torch.int32, device="cuda")
+    got = binding.parallax_varlen_prefill(pack(q), pack(r), pack(k), pack(v), cu,
+                                          out_dtype=torch.float32)
+    # same tiles, same arithmetic: identical bits
+    assert torch.equal(got, pack(dense))
+
+
+def test_varlen_malformed_lengths_are_clamped():
+    lens = [50, 70]
+    q, r, k, v, cu = make(lens, 2, 2, 64, seed=420)
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    out = torch.full_like(q, 7.0)
+    bad = torch.tensor([0, 90, 60], dtype=torch.int32, device="cuda")  # decreasing pair
+    binding.parallax_varlen_prefill(q, r, k, v, bad, 90, out=out, workspace=ws)
+    assert status_bits(ws) & 2
+    # the first sequence (rows 0..89) is computed; the clamped-empty second
+    # sequence writes nothing
+    want = oracle.parallax_varlen_prefill(q[:90], r[:90], k[:90], v[:90],
+                                          np.array([0, 90]), 64 ** -0.5)
+    assert scaled_error(out[:90], want) <= 2e-2
+    assert torch.all(out[90:] == 7.0)
+    # a max_seqlen that leaves a sequence's query tiles out is flagged too
+    q, r, k, v, cu = make([50, 200], 2, 2, 64, seed=421)
+    binding.parallax_varlen_prefill(q, r, k, v, cu, 100, workspace=ws)
+    assert status_bits(ws) & 2
+    binding.parallax_varlen_prefill(q, r, k, v, cu, 200, workspace=ws)
+    assert status_bits(ws) == 0
