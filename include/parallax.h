@@ -180,6 +180,53 @@ int parallax_decode_phase(int phase, int probe, const void* q, const void* r,
                           void* workspace, size_t workspace_bytes);
 
 /*
+ * Decode over a paged KV cache: the pages' decode (parallax-kernel 0.1.0
+ * README, "Decoding (CuTeDSL)") with its (B, kv_len, H, D) cache cut into
+ * fixed-size pages, the layout serving engines keep their caches in.
+ *  - k_pages, v_pages [num_pages][page_size][Hkv][D] bf16 (a pool of pages);
+ *    block_table [B][max_pages_per_seq] int32: key i of sequence b is slot
+ *    i % page_size of page block_table[b][i / page_size]. Only the entries a
+ *    sequence's length reaches are read.
+ *  - page_size a multiple of 64 (every 64-key tile lies in one page);
+ *    max_pages_per_seq * page_size plays the role of Lmax (cache_seqlens are
+ *    clamped to it; NULL lengths mean that many keys).
+ *  - A page id outside [0, num_pages) is not read: its keys are left out and
+ *    PARALLAX_DEVICE_STATUS_SEQLEN_CLAMPED is set.
+ *  - probe != 0: the Parallax output (r required); probe == 0: R = 0 softmax.
+ *  - bf16 inputs only; query heads per kv head at most 4 (probe) or 8.
+ *  - Workspace: parallax_decode_workspace_bytes(B, Hq, Hkv, D,
+ *    max_pages_per_seq * page_size, num_splits). Other rules as parallax_decode.
+ */
+int parallax_decode_paged(const void* q, const void* r, const void* k_pages, const void* v_pages,
+                          const int32_t* block_table, const int32_t* cache_seqlens, void* out,
+                          int B, int Hq, int Hkv, int D, float scale, void* stream, int num_pages,
+                          int page_size, int max_pages_per_seq, int probe, int out_dtype,
+                          int num_splits, void* workspace, size_t workspace_bytes);
+
+/*
+ * Block-sparse decode: parallax-kernel 0.1.0 README (opening section) notes
+ * that block sparsity is structurally compatible with Parallax. Sequence b
+ * attends only the listed 64-key blocks of its cache row: block_ids
+ * [B][max_blocks] int32, the first num_blocks[b] entries used; block j holds
+ * cache keys 64 j .. 64 j + 63, of which those below cache_seqlens[b] count.
+ * The weights are the softmax over the selected keys only; the output is the
+ * Parallax output over that key set (zero if it is empty).
+ *  - Cache as parallax_decode_ex (kv_layout BHSD or BSHD, Lmax keys per row).
+ *  - A block id outside [0, ceil(Lmax / 64)) or a count outside [0,
+ *    max_blocks] is clamped away and sets PARALLAX_DEVICE_STATUS_SEQLEN_CLAMPED.
+ *  - A block listed twice is attended twice (its keys count twice).
+ *  - bf16 inputs only; query heads per kv head at most 4 (probe) or 8.
+ *  - Workspace: parallax_decode_workspace_bytes(B, Hq, Hkv, D, 64 * max_blocks,
+ *    num_splits). Other rules as parallax_decode.
+ */
+int parallax_decode_block_sparse(const void* q, const void* r, const void* k_cache,
+                                 const void* v_cache, const int32_t* cache_seqlens,
+                                 const int32_t* block_ids, const int32_t* num_blocks, void* out,
+                                 int B, int Hq, int Hkv, int D, float scale, void* stream, int Lmax,
+                                 int kv_layout, int max_blocks, int probe, int out_dtype,
+                                 int num_splits, void* workspace, size_t workspace_bytes);
+
+/*
  * The training-shape (prefill) forward: parallax-kernel 0.1.0 README,
  * "Training (Triton)": parallax_func(q, r, k, v) maps (B, H, L, D) to
  * (B, H, L, D), causal. Row i of query head h is the decode output above over

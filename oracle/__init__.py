@@ -147,6 +147,60 @@ class Oracle:
             out[a:e] = o[0].transpose(1, 0, 2)
         return out
 
+    def _decode(self, q, r, k, v, n, scale, probe):
+        if probe:
+            return self.parallax_covariance(q, r, k, v, n, scale)
+        return self.softmax_decode(q, k, v, n, scale)
+
+    def parallax_decode_paged(self, q, r, k_pages, v_pages, block_table, seqlens, scale,
+                              probe=True):
+        """Decode over a paged cache: k_pages, v_pages [num_pages, page_size,
+        Hkv, D]; key i of sequence b is slot i % page_size of page
+        block_table[b][i // page_size]. The pages are gathered into a
+        [B, Hkv, Lmax, D] cache and the decode above runs on it."""
+        q, kp, vp = _f64(q), _f64(k_pages), _f64(v_pages)
+        r = _f64(r) if probe else np.zeros_like(q)
+        table = np.asarray(block_table.cpu() if hasattr(block_table, "cpu") else block_table)
+        B, Hq, D = q.shape
+        _, ps, Hkv, _ = kp.shape
+        Lmax = table.shape[1] * ps
+        n = (np.full(B, Lmax) if seqlens is None else
+             np.asarray(seqlens.cpu() if hasattr(seqlens, "cpu") else seqlens)).astype(np.int32)
+        k = np.zeros((B, Hkv, Lmax, D))
+        v = np.zeros((B, Hkv, Lmax, D))
+        for b in range(B):
+            for i in range(int(n[b])):
+                page, slot = table[b, i // ps], i % ps
+                k[b, :, i] = kp[page, slot]
+                v[b, :, i] = vp[page, slot]
+        return self._decode(q, r, k, v, n, scale, probe)
+
+    def parallax_decode_block_sparse(self, q, r, k, v, block_ids, num_blocks, seqlens, scale,
+                                     probe=True):
+        """Decode over the listed 64-key blocks of each cache row: the keys of
+        blocks block_ids[b][:num_blocks[b]] below seqlens[b], in list order,
+        gathered into a dense cache with per-row lengths (k, v [B, Hkv, Lmax, D])."""
+        q, k, v = _f64(q), _f64(k), _f64(v)
+        r = _f64(r) if probe else np.zeros_like(q)
+        ids = np.asarray(block_ids.cpu() if hasattr(block_ids, "cpu") else block_ids)
+        cnt = np.asarray(num_blocks.cpu() if hasattr(num_blocks, "cpu") else num_blocks)
+        B, Hkv, Lmax, D = k.shape
+        n = (np.full(B, Lmax) if seqlens is None else
+             np.asarray(seqlens.cpu() if hasattr(seqlens, "cpu") else seqlens)).astype(np.int64)
+        rows = []
+        for b in range(B):
+            keys = [key for blk in ids[b, :int(cnt[b])]
+                    for key in range(64 * int(blk), 64 * int(blk) + 64) if key < n[b]]
+            rows.append(keys)
+        width = max(1, max(len(x) for x in rows))
+        kg = np.zeros((B, Hkv, width, D))
+        vg = np.zeros((B, Hkv, width, D))
+        for b, keys in enumerate(rows):
+            kg[b, :, :len(keys)] = k[b][:, keys]
+            vg[b, :, :len(keys)] = v[b][:, keys]
+        lens = np.array([len(x) for x in rows], dtype=np.int32)
+        return self._decode(q, r, kg, vg, lens, scale, probe)
+
     # The default used by parity checks: the definition (covariance) form.
     def parallax_decode(self, q, r, k, v, seqlens, scale):
         return self.parallax_covariance(q, r, k, v, seqlens, scale)
@@ -191,6 +245,14 @@ def parallax_prefill(*a, **kw):
 
 def parallax_varlen_prefill(*a, **kw):
     return default().parallax_varlen_prefill(*a, **kw)
+
+
+def parallax_decode_paged(*a, **kw):
+    return default().parallax_decode_paged(*a, **kw)
+
+
+def parallax_decode_block_sparse(*a, **kw):
+    return default().parallax_decode_block_sparse(*a, **kw)
 
 
 def num_threads() -> int:

@@ -43,6 +43,9 @@ def load_library():
     lib.parallax_softmax_decode.argtypes = [vp, vp, vp, vp, vp] + decode_tail
     lib.parallax_decode_phase.argtypes = [i, i, vp, vp, vp, vp, vp, vp] + decode_tail
     lib.parallax_decode_ex.argtypes = [vp, vp, vp, vp, vp, vp] + decode_tail + [i, i, i, i]
+    lib.parallax_decode_paged.argtypes = [vp] * 7 + [i, i, i, i, f, vp, i, i, i, i, i, i, vp, sz]
+    lib.parallax_decode_block_sparse.argtypes = ([vp] * 8 + [i, i, i, i, f, vp, i, i, i, i, i, i,
+                                                             vp, sz])
     lib.parallax_decode_workspace_bytes.argtypes = [i, i, i, i, i, i]
     lib.parallax_decode_workspace_bytes.restype = sz
     lib.parallax_choose_splits.argtypes = [i, i, i, i]
@@ -50,7 +53,8 @@ def load_library():
     lib.parallax_status_string.argtypes = [i]
     lib.parallax_status_string.restype = ctypes.c_char_p
     for fn in (lib.parallax_decode, lib.parallax_softmax_decode, lib.parallax_decode_phase,
-               lib.parallax_decode_ex, lib.parallax_choose_splits,
+               lib.parallax_decode_ex, lib.parallax_choose_splits, lib.parallax_decode_paged,
+               lib.parallax_decode_block_sparse,
                lib.parallax_workspace_status):
         fn.restype = i
     _lib = lib
@@ -272,6 +276,78 @@ def parallax_decode_ex(q, r, k_cache, v_cache, cache_seqlens, out, workspace: Wo
         _DTYPE_CODE[q.dtype], _DTYPE_CODE[out.dtype], int(num_splits), workspace.ptr(),
         workspace.nbytes, int(bool(probe)), KV_LAYOUTS[kv_layout], int(window), int(phases))
     _check(rc, "parallax_decode_ex")
+    return out
+
+
+def _check_int32(name, t, dim):
+    if (t is None or not t.is_cuda or t.dtype != torch.int32 or t.dim() != dim
+            or not t.is_contiguous()):
+        raise ValueError(f"{name} must be a contiguous {dim}-D int32 CUDA tensor")
+
+
+def parallax_decode_paged(q, r, k_pages, v_pages, block_table, cache_seqlens=None,
+                          scale: Optional[float] = None, out=None, out_dtype=None,
+                          workspace: Optional[Workspace] = None, num_splits: int = 0,
+                          probe: bool = True, stream=None):
+    """Decode over a paged cache: k_pages, v_pages [num_pages, page_size, Hkv, D]
+    bf16, block_table int32 [B, max_pages_per_seq] (page ids per sequence),
+    cache_seqlens int32 [B] or None (every sequence fills its table)."""
+    for name, t in (("q", q), ("k_pages", k_pages), ("v_pages", v_pages)):
+        if not t.is_cuda or not t.is_contiguous() or t.dtype != torch.bfloat16:
+            raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor")
+    if q.dim() != 3 or k_pages.dim() != 4 or v_pages.shape != k_pages.shape:
+        raise ValueError("expected q [B,Hq,D] and k_pages, v_pages [num_pages,page_size,Hkv,D]")
+    B, Hq, D = q.shape
+    num_pages, page_size, Hkv, Dk = k_pages.shape
+    if Dk != D:
+        raise ValueError("head dimension of the pages does not match q")
+    _check_int32("block_table", block_table, 2)
+    if block_table.shape[0] != B:
+        raise ValueError("block_table must be [B, max_pages_per_seq]")
+    if cache_seqlens is not None:
+        _check_int32("cache_seqlens", cache_seqlens, 1)
+    max_pages = block_table.shape[1]
+    if out is None:
+        out = torch.empty((B, Hq, D), device=q.device,
+                          dtype=out_dtype if out_dtype is not None else q.dtype)
+    if workspace is None:
+        workspace = Workspace(B, Hq, Hkv, D, max_pages * page_size, num_splits, device=q.device)
+    scale = D ** -0.5 if scale is None else scale
+    rc = load_library().parallax_decode_paged(
+        q.data_ptr(), _ptr(r) if probe else None, k_pages.data_ptr(), v_pages.data_ptr(),
+        block_table.data_ptr(), _ptr(cache_seqlens), out.data_ptr(), B, Hq, Hkv, D, float(scale),
+        _stream(stream), num_pages, page_size, max_pages, int(bool(probe)), _DTYPE_CODE[out.dtype],
+        int(num_splits), workspace.ptr(), workspace.nbytes)
+    _check(rc, "parallax_decode_paged")
+    return out
+
+
+def parallax_decode_block_sparse(q, r, k_cache, v_cache, block_ids, num_blocks,
+                                 cache_seqlens=None, scale: Optional[float] = None, out=None,
+                                 out_dtype=None, workspace: Optional[Workspace] = None,
+                                 num_splits: int = 0, probe: bool = True, kv_layout: str = "bhsd",
+                                 stream=None):
+    """Decode over the listed 64-key blocks of each sequence: block_ids int32
+    [B, max_blocks] (first num_blocks[b] used), num_blocks int32 [B]."""
+    B, Hq, Hkv, D, Lmax = _shapes(q, k_cache, v_cache, cache_seqlens, kv_layout)
+    _check_int32("block_ids", block_ids, 2)
+    _check_int32("num_blocks", num_blocks, 1)
+    if block_ids.shape[0] != B or num_blocks.shape != (B,):
+        raise ValueError("block_ids must be [B, max_blocks] and num_blocks [B]")
+    max_blocks = block_ids.shape[1]
+    if out is None:
+        out = torch.empty((B, Hq, D), device=q.device,
+                          dtype=out_dtype if out_dtype is not None else q.dtype)
+    if workspace is None:
+        workspace = Workspace(B, Hq, Hkv, D, 64 * max_blocks, num_splits, device=q.device)
+    scale = D ** -0.5 if scale is None else scale
+    rc = load_library().parallax_decode_block_sparse(
+        q.data_ptr(), _ptr(r) if probe else None, k_cache.data_ptr(), v_cache.data_ptr(),
+        _ptr(cache_seqlens), block_ids.data_ptr(), num_blocks.data_ptr(), out.data_ptr(), B, Hq,
+        Hkv, D, float(scale), _stream(stream), Lmax, KV_LAYOUTS[kv_layout], max_blocks,
+        int(bool(probe)), _DTYPE_CODE[out.dtype], int(num_splits), workspace.ptr(),
+        workspace.nbytes)
+    _check(rc, "parallax_decode_block_sparse")
     return out
 
 

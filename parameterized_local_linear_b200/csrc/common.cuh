@@ -29,6 +29,12 @@ struct DecodeParams {
   float scale_log2;       // qk_scale * log2(e): logits are kept in the log2 domain
   unsigned long long timeout_ns;  // bound of every wait inside the kernels
   int debug_skip_first_tile;      // testing hook: the producer never fills stage 0
+  // where the keys of a row come from (partition.cuh, KvMode)
+  int kv_mode;
+  const int32_t* table;   // paged: [B][table_stride] page ids; block-sparse: block ids
+  int table_stride;
+  const int32_t* num_blocks;  // block-sparse: [B] listed blocks
+  int page_size, num_pages;   // paged
 };
 
 // ------------------------------------------------ TMA kernel geometry ------
@@ -65,7 +71,7 @@ __host__ __device__ inline TcSmemLayout tc_smem_layout(int D, int stage_bytes, i
   L.off_bar = align_up(L.off_merge + kConsumerWarps * G * rec_floats(D) * 4, 16);
   // full[stages], empty[stages], fin[2]
   L.off_misc = L.off_bar + 8 * (2 * stages + 2);
-  L.total = L.off_misc + 16 + 1024;  // abort flag, alignment slack
+  L.total = L.off_misc + 48 + 1024;  // abort flag, per-stage valid keys, alignment slack
   return L;
 }
 

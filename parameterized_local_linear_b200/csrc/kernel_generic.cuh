@@ -40,7 +40,7 @@ __global__ void __launch_bounds__(kGenericThreads)
 
   pdl_wait_primary();  // launched with programmatic stream serialisation
   const PartitionInfo part =
-      locate_partition(p.seqlens, p.B, p.Hkv, p.Lmax, p.window, blockIdx.x, gridDim.x);
+      locate_partition(key_space(p), p.B, p.Hkv, blockIdx.x, gridDim.x);
   if (blockIdx.x == 0 && threadIdx.x == 0 && part.clamped) atomicOr(p.status, 2u);
   pdl_launch_dependents();
   if (part.lo >= part.hi) return;
@@ -52,7 +52,7 @@ __global__ void __launch_bounds__(kGenericThreads)
   const int tid = threadIdx.x, D = p.D, G = p.G, REC = rec_floats(D);
 
   PieceCursor cur;
-  cur.init(part, p.seqlens, p.B, p.Hkv, p.Lmax, p.window);
+  cur.init(part, key_space(p), p.B, p.Hkv);
   Piece pc;
   while (cur.next(pc)) {
     const long long kv0 = pc.b * p.kv_sb + pc.g * p.kv_sh + pc.kbase * p.kv_sk;

@@ -41,13 +41,13 @@ __global__ void __launch_bounds__(kMergeThreads, 4) parallax_merge_kernel(const 
   const float kNegInf = __int_as_float(0xff800000u);
   const int tid = threadIdx.x;
   const int c = blockIdx.x, P = gridDim.x;
-  const PartitionInfo part = locate_partition(p.seqlens, p.B, p.Hkv, p.Lmax, p.window, c, P);
+  const PartitionInfo part = locate_partition(key_space(p), p.B, p.Hkv, c, P);
 
   // Sequences without keys: zero output (nothing else writes these rows).
   if (blockIdx.y == 0) {
     for (int b = c; b < p.B; b += P) {
       int kb;
-      if (attended_keys(p.seqlens, b, p.Lmax, p.window, &kb) != 0) continue;
+      if (item_keys(key_space(p), b, &kb) != 0) continue;
       for (int idx = tid; idx < p.Hq * p.D; idx += kMergeThreads) {
         const size_t oi = (size_t)b * p.Hq * p.D + idx;
         if (OUT_F32)
@@ -117,7 +117,8 @@ __global__ void __launch_bounds__(kMergeThreads, 4) parallax_merge_kernel(const 
 #pragma unroll
     for (int k = 0; k < kMergeChunk; ++k) {
       if (k < nch) {
-        const float w = ex2_approx(s_m[k * G + h_col] - M_new);
+        const float mk = s_m[k * G + h_col];
+        const float w = mk == kNegInf ? 0.f : ex2_approx(mk - M_new);  // a piece with no key
         sum.x += w * v[k].x;
         sum.y += w * v[k].y;
         sum.z += w * v[k].z;
@@ -137,7 +138,7 @@ __global__ void __launch_bounds__(kMergeThreads, 4) parallax_merge_kernel(const 
   }
   // Output: the A-column thread writes its 4 dimensions; with the probe the C
   // column is the next thread.
-  const float inv = 1.f / L_run;
+  const float inv = L_run > 0.f ? 1.f / L_run : 0.f;  // no attended key: o = 0
   float4 o = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
   if (PROBE) {
     const float cx = __shfl_down_sync(0xffffffffu, acc.x, 1);

@@ -42,6 +42,30 @@
 
 namespace plx {
 
+// Paged and block-sparse rows: where logical tile k0 (a multiple of 64) of
+// batch row b lives, as (*key, *item) coordinates of the K/V tensor maps, and
+// how many of its keys are attended (*nv, a prefix of the tile). An id outside
+// the pool or the cache gives an empty tile and sets the clamped status bit.
+__device__ __forceinline__ void tile_source(const DecodeParams& p, int b, int k0, int* key,
+                                            int* item, int* nv) {
+  const int n = p.seqlens ? clamp_len(__ldg(p.seqlens + b), p.Lmax) : p.Lmax;
+  if (p.kv_mode == kKvPaged) {
+    const int page = __ldg(p.table + (size_t)b * p.table_stride + k0 / p.page_size);
+    const bool ok = page >= 0 && page < p.num_pages;
+    *key = ok ? k0 % p.page_size : 0;
+    *item = ok ? page : 0;
+    *nv = ok ? max(0, min(kTileKeys, n - k0)) : 0;
+    if (!ok) atomicOr(p.status, 2u /* PARALLAX_DEVICE_STATUS_SEQLEN_CLAMPED */);
+  } else {  // block-sparse: the listed block of the cache row
+    const int blk = __ldg(p.table + (size_t)b * p.table_stride + k0 / kTileKeys);
+    const bool ok = blk >= 0 && (long long)blk * kTileKeys < p.Lmax;
+    *key = ok ? blk * kTileKeys : 0;
+    *item = b;
+    *nv = ok ? max(0, min(kTileKeys, n - blk * kTileKeys)) : 0;
+    if (!ok) atomicOr(p.status, 2u);
+  }
+}
+
 template <int D, bool PROBE, bool OUT_F32, bool PSPLIT>
 __global__ void __launch_bounds__(kTcThreads, 1)
     parallax_tc_kernel(const __grid_constant__ CUtensorMap tmK,
@@ -64,6 +88,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t bar_empty = bar_full + 8 * kStages;
   const uint32_t bar_fin = bar_empty + 8 * kStages;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L.off_misc);
+  // paged / block-sparse rows: valid keys (a prefix) of the tile in each stage
+  volatile int* stage_valid = reinterpret_cast<volatile int*>(gbase + L.off_misc + 16);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
@@ -86,7 +112,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // the previous kernel in the stream; nothing below may run before it ends.
   pdl_wait_primary();
   const PartitionInfo part =
-      locate_partition(p.seqlens, p.B, p.Hkv, p.Lmax, p.window, blockIdx.x, gridDim.x);
+      locate_partition(key_space(p), p.B, p.Hkv, blockIdx.x, gridDim.x);
   if (blockIdx.x == 0 && tid == 0 && part.clamped)
     atomicOr(p.status, 2u /* PARALLAX_DEVICE_STATUS_SEQLEN_CLAMPED */);
   // The merge grid may be scheduled once every CTA has its first stage in
@@ -100,7 +126,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (warp == kConsumerWarps) {
     if (lane != 0) return;
     PieceCursor cur;
-    cur.init(part, p.seqlens, p.B, p.Hkv, p.Lmax, p.window);
+    cur.init(part, key_space(p), p.B, p.Hkv);
     Piece pc;
     int stage = 0;
     uint32_t ph = 0, issued_mask = 0, issued_par = 0;
@@ -116,10 +142,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         } else {
           const uint32_t full = bar_full + 8 * stage;
           const uint32_t sK = base + stage * kStageBytes;
+          // source of the tile: (key or page slot, batch row or page) on the maps
+          int key = pc.kbase + k0, item = pc.b;
+          if (p.kv_mode != kKvContiguous) {
+            int nv;
+            tile_source(p, pc.b, k0, &key, &item, &nv);
+            stage_valid[stage] = nv;  // published by the arrive below
+          }
           mbar_arrive_expect_tx(full, kStageBytes);
-          const int key = pc.kbase + k0;  // cache position of the tile's first key
-          tma_load_5d(sK, &tmK, 0, key, 0, pc.g, pc.b, full, policy);
-          tma_load_5d(sK + kKBytes, &tmV, 0, key, 0, pc.g, pc.b, full, policy);
+          tma_load_5d(sK, &tmK, 0, key, 0, pc.g, item, full, policy);
+          tma_load_5d(sK + kKBytes, &tmV, 0, key, 0, pc.g, item, full, policy);
           if (issued_mask == 0) pdl_launch_dependents();
           issued_mask |= 1u << stage;
           issued_par = (issued_par & ~(1u << stage)) | (ph << stage);
@@ -160,7 +192,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int sw = lane & 7;  // row index mod 8 = the 128-byte swizzle phase of both rows
 
   PieceCursor cur;
-  cur.init(part, p.seqlens, p.B, p.Hkv, p.Lmax, p.window);
+  cur.init(part, key_space(p), p.B, p.Hkv);
   Piece pc;
   int stage = 0;
   uint32_t ph = 0, fph = 0;
@@ -206,7 +238,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         pdl_launch_dependents();
         triggered = true;
       }
-      const int nvalid = min(kTileKeys, pc.i + pc.len - k0);
+      const int nvalid = p.kv_mode == kKvContiguous ? min(kTileKeys, pc.i + pc.len - k0)
+                                                    : stage_valid[stage];
       const uint32_t sK = base + stage * kStageBytes;
       const uint32_t sV = sK + kKBytes;
       if (my0 < nvalid) {
@@ -439,7 +472,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
         }
         if (pc.complete) {
-          const float inv = 1.f / Lw;
+          const float inv = Lw > 0.f ? 1.f / Lw : 0.f;  // no attended key: o = 0
           const float vbar = Aw * inv;
           const float o = PROBE ? vbar + Cw * inv - (Bw * inv) * vbar : vbar;
           const size_t oi = ((size_t)pc.b * p.Hq + (size_t)pc.g * G + h) * D + d;

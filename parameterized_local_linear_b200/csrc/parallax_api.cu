@@ -42,6 +42,12 @@ struct Call {
   int kv_layout, window;
   unsigned long long timeout_ns;
   int debug_skip_first_tile;
+  // paged / block-sparse rows (partition.cuh, KvMode)
+  int kv_mode;
+  const int32_t* table;  // page ids or block ids, [B][table_stride]
+  int table_stride;
+  const int32_t* num_blocks;
+  int page_size, num_pages;
 };
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -97,8 +103,32 @@ int resolve_splits(int num_splits, int B, int Hkv, int Lmax, int* P) {
   return PARALLAX_OK;
 }
 
+// Keys per row the partition heuristic plans for.
+int planned_len(const Call& c) {
+  if (c.kv_mode == kKvPaged) return c.table_stride * c.page_size;
+  if (c.kv_mode == kKvBlockSparse) return c.table_stride * kTileKeys;
+  return effective_len(c.Lmax, c.window);
+}
+
 int validate(const Call& c) {
   if (!c.q || !c.k || !c.v || !c.out || !c.ws) return PARALLAX_ERR_NULL_POINTER;
+  if (c.kv_mode != kKvContiguous) {
+    if (!c.table || (c.kv_mode == kKvBlockSparse && !c.num_blocks)) return PARALLAX_ERR_NULL_POINTER;
+    if ((reinterpret_cast<uintptr_t>(c.table) & 3u) ||
+        (reinterpret_cast<uintptr_t>(c.num_blocks) & 3u))
+      return PARALLAX_ERR_MISALIGNED;
+    if (c.table_stride < 1 || c.window != 0) return PARALLAX_ERR_BAD_SHAPE;
+    if (c.kv_mode == kKvPaged &&
+        (c.page_size < kTileKeys || c.page_size % kTileKeys != 0 || c.num_pages < 1 ||
+         (long long)c.table_stride * c.page_size > 0x7fffffffLL))
+      return PARALLAX_ERR_BAD_SHAPE;
+    if (c.kv_mode == kKvBlockSparse && (long long)c.table_stride * kTileKeys > 0x7fffffffLL)
+      return PARALLAX_ERR_BAD_SHAPE;
+    // these rows are served by the TMA kernel only: bf16 inputs, a group that fits it
+    const int G = c.Hkv > 0 ? c.Hq / c.Hkv : 0;
+    if (c.in_dtype != PARALLAX_DTYPE_BF16) return PARALLAX_ERR_UNSUPPORTED_DTYPE;
+    if (c.probe ? 2 * G > 8 : G > 8) return PARALLAX_ERR_BAD_SHAPE;
+  }
   if (c.probe && !c.r) return PARALLAX_ERR_NULL_POINTER;
   if (!shape_ok(c.B, c.Hq, c.Hkv, c.D, c.Lmax)) return PARALLAX_ERR_BAD_SHAPE;
   if ((c.kv_layout != PARALLAX_KV_BHSD && c.kv_layout != PARALLAX_KV_BSHD) || c.window < 0)
@@ -184,10 +214,13 @@ int launch_tc(const Call& c, const DecodeParams& prm, int P) {
   int st = set_smem_once(kernel, L.total, done);
   if (st != PARALLAX_OK) return st;
   CUtensorMap tmK, tmV;
-  if ((st = encode_cache_map(&tmK, c.k, D, c.Lmax, c.Hkv, c.B, c.kv_layout)) != PARALLAX_OK)
-    return st;
-  if ((st = encode_cache_map(&tmV, c.v, D, c.Lmax, c.Hkv, c.B, c.kv_layout)) != PARALLAX_OK)
-    return st;
+  // paged: the page pool [num_pages][page_size][Hkv][D] is a cache of num_pages
+  // rows of page_size keys in the (B, L, H, D) layout
+  const bool paged = c.kv_mode == kKvPaged;
+  const int rows = paged ? c.num_pages : c.B, len = paged ? c.page_size : c.Lmax;
+  const int layout = paged ? PARALLAX_KV_BSHD : c.kv_layout;
+  if ((st = encode_cache_map(&tmK, c.k, D, len, c.Hkv, rows, layout)) != PARALLAX_OK) return st;
+  if ((st = encode_cache_map(&tmV, c.v, D, len, c.Hkv, rows, layout)) != PARALLAX_OK) return st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
@@ -259,8 +292,7 @@ int run(const Call& c) {
   int st = validate(c);
   if (st != PARALLAX_OK) return st;
   int P = 0;
-  if ((st = resolve_splits(c.num_splits, c.B, c.Hkv, effective_len(c.Lmax, c.window), &P)) !=
-      PARALLAX_OK)
+  if ((st = resolve_splits(c.num_splits, c.B, c.Hkv, planned_len(c), &P)) != PARALLAX_OK)
     return st;
   const int G = c.Hq / c.Hkv;
   if (c.ws_bytes < workspace_bytes_for(G, c.D, P)) return PARALLAX_ERR_WORKSPACE_TOO_SMALL;
@@ -284,7 +316,13 @@ int run(const Call& c) {
   prm.Hkv = c.Hkv;
   prm.G = G;
   prm.D = c.D;
-  prm.Lmax = c.Lmax;
+  prm.Lmax = c.kv_mode == kKvPaged ? c.table_stride * c.page_size : c.Lmax;
+  prm.kv_mode = c.kv_mode;
+  prm.table = c.table;
+  prm.table_stride = c.table_stride;
+  prm.num_blocks = c.num_blocks;
+  prm.page_size = c.page_size;
+  prm.num_pages = c.num_pages;
   prm.scale_log2 = (float)((double)c.scale * 1.4426950408889634);  // log2(e)
   prm.timeout_ns = c.timeout_ns;
   prm.debug_skip_first_tile = c.debug_skip_first_tile;
@@ -323,6 +361,12 @@ Call make_call(int phases, bool probe, const void* q, const void* r, const void*
   c.window = 0;
   c.timeout_ns = kDefaultTimeoutNs;
   c.debug_skip_first_tile = 0;
+  c.kv_mode = kKvContiguous;
+  c.table = nullptr;
+  c.table_stride = 0;
+  c.num_blocks = nullptr;
+  c.page_size = 0;
+  c.num_pages = 0;
   return c;
 }
 
@@ -374,6 +418,42 @@ int parallax_decode_ex(const void* q, const void* r, const void* k_cache, const 
                      workspace_bytes);
   c.kv_layout = kv_layout;
   c.window = window;
+  return run(c);
+}
+
+int parallax_decode_paged(const void* q, const void* r, const void* k_pages, const void* v_pages,
+                          const int32_t* block_table, const int32_t* cache_seqlens, void* out,
+                          int B, int Hq, int Hkv, int D, float scale, void* stream, int num_pages,
+                          int page_size, int max_pages_per_seq, int probe, int out_dtype,
+                          int num_splits, void* workspace, size_t workspace_bytes) {
+  if (page_size < 1 || max_pages_per_seq < 1) return PARALLAX_ERR_BAD_SHAPE;
+  const long long lmax = (long long)page_size * max_pages_per_seq;
+  if (lmax > 0x7fffffffLL) return PARALLAX_ERR_BAD_SHAPE;
+  Call c = make_call(3, probe != 0, q, r, k_pages, v_pages, cache_seqlens, out, B, Hq, Hkv, D,
+                     scale, stream, (int)lmax, PARALLAX_DTYPE_BF16, out_dtype, num_splits,
+                     workspace, workspace_bytes);
+  c.kv_mode = kKvPaged;
+  c.table = block_table;
+  c.table_stride = max_pages_per_seq;
+  c.page_size = page_size;
+  c.num_pages = num_pages;
+  return run(c);
+}
+
+int parallax_decode_block_sparse(const void* q, const void* r, const void* k_cache,
+                                 const void* v_cache, const int32_t* cache_seqlens,
+                                 const int32_t* block_ids, const int32_t* num_blocks, void* out,
+                                 int B, int Hq, int Hkv, int D, float scale, void* stream, int Lmax,
+                                 int kv_layout, int max_blocks, int probe, int out_dtype,
+                                 int num_splits, void* workspace, size_t workspace_bytes) {
+  Call c = make_call(3, probe != 0, q, r, k_cache, v_cache, cache_seqlens, out, B, Hq, Hkv, D,
+                     scale, stream, Lmax, PARALLAX_DTYPE_BF16, out_dtype, num_splits, workspace,
+                     workspace_bytes);
+  c.kv_layout = kv_layout;
+  c.kv_mode = kKvBlockSparse;
+  c.table = block_ids;
+  c.table_stride = max_blocks;
+  c.num_blocks = num_blocks;
   return run(c);
 }
 

@@ -23,16 +23,57 @@ __device__ __forceinline__ int clamp_len(int n, int Lmax) {
   return n < 0 ? 0 : (n > Lmax ? Lmax : n);
 }
 
-// The attended keys of batch row b: its clamped length n (every row holds Lmax
-// keys when there is no length array), and with a sliding window of W > 0
-// only the last min(n, W) of them. Returns that count; *kbase gets the first
-// attended key, n - count.
-__device__ __forceinline__ int attended_keys(const int32_t* __restrict__ seqlens, int b, int Lmax,
-                                             int window, int* kbase) {
-  const int n = seqlens ? clamp_len(__ldg(seqlens + b), Lmax) : Lmax;
-  const int ne = (window > 0 && n > window) ? window : n;
+// Where the keys of each batch row come from.
+//   kKvContiguous  the cache row itself: keys 0..n-1 (with a sliding window
+//                  W > 0 only the last min(n, W)).
+//   kKvPaged       fixed-size pages listed per row in a block table: key i is
+//                  slot i % page_size of page table[b][i / page_size].
+//   kKvBlockSparse a per-row list of 64-key blocks of the cache row: logical
+//                  tile t is cache keys 64 table[b][t] .. +63 (keys >= n masked).
+// The paged and block-sparse rows are walked in whole 64-key tiles, so every
+// tile a CTA loads sits inside one page or block.
+enum KvMode { kKvContiguous = 0, kKvPaged = 1, kKvBlockSparse = 2 };
+
+struct KeySpace {
+  const int32_t* seqlens;     // [B], or NULL: every row holds Lmax keys
+  const int32_t* num_blocks;  // block-sparse: [B] listed blocks per row
+  int Lmax, window, mode, max_blocks;
+};
+
+// The keys batch row b contributes to the end-to-end key sequence the
+// partitions cut, and (contiguous rows) *kbase = the cache position of the
+// first one. Paged rows count their n keys rounded up to whole tiles and
+// block-sparse rows 64 per listed block; the kernels mask the keys past n.
+__device__ __forceinline__ int item_keys(const KeySpace& ks, int b, int* kbase) {
+  const int n = ks.seqlens ? clamp_len(__ldg(ks.seqlens + b), ks.Lmax) : ks.Lmax;
+  *kbase = 0;
+  if (ks.mode == kKvPaged) return (n + kRangeAlign - 1) / kRangeAlign * kRangeAlign;
+  if (ks.mode == kKvBlockSparse) {
+    const int nb = __ldg(ks.num_blocks + b);
+    return kRangeAlign * (nb < 0 ? 0 : (nb > ks.max_blocks ? ks.max_blocks : nb));
+  }
+  const int ne = (ks.window > 0 && n > ks.window) ? ks.window : n;
   *kbase = n - ne;
   return ne;
+}
+
+template <typename Params>
+__device__ __forceinline__ KeySpace key_space(const Params& p) {
+  return KeySpace{p.seqlens, p.num_blocks, p.Lmax, p.window, p.kv_mode, p.table_stride};
+}
+
+// A length or block count outside its range (clamped by item_keys).
+__device__ __forceinline__ bool item_clamped(const KeySpace& ks, int b) {
+  bool bad = false;
+  if (ks.seqlens) {
+    const int n = __ldg(ks.seqlens + b);
+    bad = n < 0 || n > ks.Lmax;
+  }
+  if (ks.mode == kKvBlockSparse) {
+    const int nb = __ldg(ks.num_blocks + b);
+    bad = bad || nb < 0 || nb > ks.max_blocks;
+  }
+  return bad;
 }
 
 struct PartitionInfo {
@@ -40,7 +81,7 @@ struct PartitionInfo {
   long long per;    // keys per partition
   long long lo, hi; // this partition's range
   int b, g, i;      // item and key offset at position lo (valid if lo < hi)
-  int n;            // attended keys of batch b
+  int n;            // keys of batch b (item_keys)
   int kbase;        // first attended key of batch b
   int clamped;      // some cache_seqlens value was outside [0, Lmax]
 };
@@ -50,19 +91,16 @@ struct PartitionInfo {
 // chunk of cache_seqlens (read-only path, so the re-reads hit L1), a warp scan
 // gives the prefix sums, and the lane whose chunk holds position lo walks it
 // to find the item there. c is this block's index among P partitions.
-__device__ inline PartitionInfo locate_partition(const int32_t* __restrict__ seqlens, int B,
-                                                 int Hkv, int Lmax, int window, int c, int P) {
+__device__ inline PartitionInfo locate_partition(const KeySpace& ks, int B, int Hkv, int c,
+                                                 int P) {
   const int lane = threadIdx.x & 31;
   const int chunk = (B + 31) / 32;
   const int b0 = min(B, lane * chunk), b1 = min(B, b0 + chunk);
   long long local = 0;
   int clamped = 0, kb;
   for (int b = b0; b < b1; ++b) {
-    if (seqlens) {
-      const int n = __ldg(seqlens + b);
-      clamped |= (n < 0 || n > Lmax);
-    }
-    local += attended_keys(seqlens, b, Lmax, window, &kb);
+    clamped |= item_clamped(ks, b);
+    local += item_keys(ks, b, &kb);
   }
   long long incl = local;  // inclusive scan over lanes
 #pragma unroll
@@ -86,7 +124,7 @@ __device__ inline PartitionInfo locate_partition(const int32_t* __restrict__ seq
   long long within = 0;
   if (p.lo < p.hi && p.lo >= pos && p.lo < pos + (long long)Hkv * local) {
     for (int b = b0; b < b1; ++b) {
-      const int n = attended_keys(seqlens, b, Lmax, window, &kb);
+      const int n = item_keys(ks, b, &kb);
       const long long blk = (long long)Hkv * n;
       if (p.lo < pos + blk) {
         fb = b;
@@ -122,13 +160,12 @@ struct Piece {
 
 // Walks the pieces of one partition; every role of a CTA walks the same list.
 struct PieceCursor {
-  int b, g, i, n, kbase;  // n, kbase: attended keys of batch b and the first one
+  int b, g, i, n, kbase;  // n, kbase: keys of batch b (item_keys) and the first one
   long long pos, lo, hi;
-  const int32_t* seqlens;
-  int B, Hkv, Lmax, window;
+  KeySpace ks;
+  int B, Hkv;
 
-  __device__ void init(const PartitionInfo& p, const int32_t* sl, int B_, int Hkv_, int Lmax_,
-                       int window_) {
+  __device__ void init(const PartitionInfo& p, const KeySpace& ks_, int B_, int Hkv_) {
     b = p.b;
     g = p.g;
     i = p.i;
@@ -137,11 +174,9 @@ struct PieceCursor {
     pos = p.lo;
     lo = p.lo;
     hi = p.hi;
-    seqlens = sl;
+    ks = ks_;
     B = B_;
     Hkv = Hkv_;
-    Lmax = Lmax_;
-    window = window_;
   }
 
   __device__ bool next(Piece& pc) {
@@ -164,7 +199,7 @@ struct PieceCursor {
         g = 0;
         ++b;
         n = 0;
-        while (pos < hi && b < B && (n = attended_keys(seqlens, b, Lmax, window, &kbase)) == 0) ++b;
+        while (pos < hi && b < B && (n = item_keys(ks, b, &kbase)) == 0) ++b;
       }
     }
     return true;

@@ -409,6 +409,60 @@ def pin_varlen_sequences_isolated(orc):
             close(o[cu[b]], np.repeat(v[cu[b]], 2, axis=0), 1e-12, "varlen first row")
 
 
+# ------------------------------------------------------ paged, block-sparse --
+
+def pin_paged_is_the_gathered_cache(orc):
+    """Pages cut from a dense cache and scattered through the pool under a
+    random table give the dense decode; with r = 0, torch's softmax attention."""
+    q, r, k, v, n = rand_case(40, B=2, Hq=4, Hkv=2, D=8, Lmax=24, lengths=(11, 24))
+    ps = 8  # small pages for the oracle (the kernel takes multiples of 64)
+    pages = k.shape[2] // ps
+    perm = np.random.default_rng(41).permutation(2 * pages)
+    table = perm.reshape(2, pages).astype(np.int32)
+    kp = np.zeros((2 * pages, ps, 2, 8))
+    vp = np.zeros_like(kp)
+    for b in range(2):
+        for j in range(pages):
+            kp[table[b, j]] = k[b, :, j * ps:(j + 1) * ps].transpose(1, 0, 2)
+            vp[table[b, j]] = v[b, :, j * ps:(j + 1) * ps].transpose(1, 0, 2)
+    got = orc.parallax_decode_paged(q, r, kp, vp, table, n, 0.3)
+    close(got, orc.parallax_decode(q, r, k, v, n, 0.3), 1e-12, "paged = dense")
+    got0 = orc.parallax_decode_paged(q, None, kp, vp, table, n, 0.3, probe=False)
+    close(got0, torch_softmax_attention(q, k, v, n, 0.3), 1e-12, "paged r=0 = softmax")
+
+
+def pin_block_sparse_selects_keys(orc):
+    """r = 0 over a block list is softmax attention restricted to those keys
+    (a boolean mask on torch's SDPA); all blocks listed is the dense decode; an
+    empty list is a zero output."""
+    rng = np.random.default_rng(42)
+    B, Hq, Hkv, D, Lmax = 2, 4, 2, 8, 256
+    q = rng.standard_normal((B, Hq, D))
+    r = rng.standard_normal((B, Hq, D)) * 0.5
+    k = rng.standard_normal((B, Hkv, Lmax, D))
+    v = rng.standard_normal((B, Hkv, Lmax, D))
+    n = np.array([200, 256], dtype=np.int32)
+    ids = np.array([[0, 3, 2, 0], [1, 3, 0, 0]], dtype=np.int32)
+    cnt = np.array([3, 2], dtype=np.int32)
+    mask = np.zeros((B, Lmax), bool)
+    for b in range(B):
+        for blk in ids[b, :cnt[b]]:
+            mask[b, 64 * blk:64 * blk + 64] = True
+    mask &= np.arange(Lmax)[None] < n[:, None]
+    qt = torch.from_numpy(q)[:, :, None]                      # [B, Hq, 1, D]
+    kt = torch.repeat_interleave(torch.from_numpy(k), 2, dim=1)
+    vt = torch.repeat_interleave(torch.from_numpy(v), 2, dim=1)
+    want = torch.nn.functional.scaled_dot_product_attention(
+        qt, kt, vt, attn_mask=torch.from_numpy(mask)[:, None, None], scale=0.3)[:, :, 0].numpy()
+    got = orc.parallax_decode_block_sparse(q, None, k, v, ids, cnt, n, 0.3, probe=False)
+    close(got, want, 1e-12, "block-sparse r=0 = masked softmax")
+    full = np.tile(np.arange(4, dtype=np.int32), (B, 1))
+    close(orc.parallax_decode_block_sparse(q, r, k, v, full, np.array([4, 4]), n, 0.3),
+          orc.parallax_decode(q, r, k, v, n, 0.3), 1e-12, "all blocks = dense")
+    empty = orc.parallax_decode_block_sparse(q, r, k, v, ids, np.array([0, 2]), n, 0.3)
+    assert np.all(empty[0] == 0.0) and np.all(np.isfinite(empty[1])), "empty block list"
+
+
 PINS = [pin_hand_examples, pin_r_zero_is_softmax, pin_single_key_returns_v,
         pin_constant_values, pin_value_shift_and_scale, pin_key_translation,
         pin_linear_in_r, pin_key_permutation, pin_forms_agree,
@@ -416,4 +470,5 @@ PINS = [pin_hand_examples, pin_r_zero_is_softmax, pin_single_key_returns_v,
         pin_empty_sequence_is_zero, pin_prefill_r_zero_is_sdpa,
         pin_prefill_first_row_and_causality, pin_prefill_local_linear_intercept,
         pin_prefill_gqa_mapping, pin_varlen_r_zero_is_masked_sdpa,
-        pin_varlen_equal_lengths_match_dense, pin_varlen_sequences_isolated]
+        pin_varlen_equal_lengths_match_dense, pin_varlen_sequences_isolated,
+        pin_paged_is_the_gathered_cache, pin_block_sparse_selects_keys]
