@@ -4,6 +4,7 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload qwen|large|long|ragged|tiny]
     python bench.py --impl reference ...   # the fp64 CPU oracle as the reference arm
     python bench.py --prefill [--prefill-shape B,Hq,Hkv,L,D]   # the causal training-shape forward
+    python bench.py --kv-mode paged|block_sparse --workload large   # paged / block-sparse decode
 
 A step is one Parallax decode pass (split-KV kernel + merge kernel) over one
 batch of synthetic input resident in HBM. The headline value is KV-read
@@ -63,10 +64,17 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="bound of the CPU oracle baseline sample (seconds)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kv-mode", choices=["contiguous", "paged", "block_sparse"],
+                    default="contiguous", help="where the decode reads its keys from")
+    ap.add_argument("--page-size", type=int, default=256)
+    ap.add_argument("--density", type=float, default=0.5,
+                    help="block-sparse: fraction of each sequence's 64-key blocks attended")
     ap.add_argument("--prefill", action="store_true",
                     help="time the causal training-shape forward instead of the decode")
     ap.add_argument("--prefill-shape", default=PREFILL_DEFAULT_SHAPE,
                     help="B,Hq,Hkv,L,D of the prefill forward")
+    ap.add_argument("--varlen", action="store_true",
+                    help="prefill: B packed sequences of seeded lengths U{1..L} instead")
     a = ap.parse_args()
     if a.prefill:
         a.steps = a.steps if a.steps is not None else 50
@@ -363,6 +371,13 @@ def run_prefill(args):
     flops = prefill_flops(B, Hq, L, D)
     cfg = {"workload": f"prefill: Parallax causal forward B={B} Hq={Hq} Hkv={Hkv} L={L} D={D} "
                        f"bf16 N(0,1)", "global_batch": B, "seq_len": L}
+    lens = None
+    if args.varlen:
+        g = torch.Generator().manual_seed(11)
+        lens = torch.randint(1, L + 1, (B,), generator=g).tolist()
+        flops = sum(8 * D * Hq * n * (n + 1) // 2 for n in lens)
+        cfg["workload"] = (f"varlen prefill: {B} packed sequences, lengths U{{1..{L}}} seeded "
+                           f"({sum(lens)} tokens), Hq={Hq} Hkv={Hkv} D={D} bf16 N(0,1)")
     if args.impl == "reference":
         if int(os.environ.get("RANK", "0")) != 0:
             return 0
@@ -385,7 +400,17 @@ def run_prefill(args):
     binding.load_library()
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.set_stream(stream)
-    q, r, k, v = prefill_inputs(B, Hq, Hkv, L, D, dev)
+    if lens is None:
+        q, r, k, v = prefill_inputs(B, Hq, Hkv, L, D, dev)
+        call = lambda: binding.parallax_prefill(q, r, k, v, out=out, workspace=ws, stream=stream)
+    else:  # the same draws, packed: [total, H, D]
+        total = sum(lens)
+        q, r, k, v = (t[0].transpose(0, 1).contiguous() for t in
+                      prefill_inputs(1, Hq, Hkv, total, D, dev))
+        cu = torch.tensor([0] + list(torch.tensor(lens).cumsum(0).tolist()), dtype=torch.int32,
+                          device=dev)
+        call = lambda: binding.parallax_varlen_prefill(q, r, k, v, cu, max(lens), out=out,
+                                                       workspace=ws, stream=stream)
     out = torch.empty_like(q)
     ws = torch.zeros(256, dtype=torch.uint8, device=dev)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
@@ -398,7 +423,7 @@ def run_prefill(args):
                 flush.fill_(float(i))
             if events:
                 events[i][0].record(stream)
-            binding.parallax_prefill(q, r, k, v, out=out, workspace=ws, stream=stream)
+            call()
             if events:
                 events[i][1].record(stream)
 
@@ -435,6 +460,9 @@ def run_prefill(args):
     # grouped heads): context for the tensor-core efficiency, not the target
     sdpa = None
     try:
+        if lens is not None:
+            raise RuntimeError("no packed-sequence SDPA in torch; see the dense line")
+
         def run_sdpa(k_steps):
             for i in range(k_steps):
                 if flush is not None:
@@ -456,7 +484,7 @@ def run_prefill(args):
         for _ in range(k_steps):
             for dst, src in ((q, hq), (r, hr), (k, hk), (v, hv)):
                 dst.copy_(src, non_blocking=True)
-            binding.parallax_prefill(q, r, k, v, out=out, workspace=ws, stream=stream)
+            call()
             out_host.copy_(out, non_blocking=True)
 
     k_e2e = min(args.steps, 20)
@@ -500,12 +528,181 @@ def run_prefill(args):
     return 0
 
 
+# -------------------------------------------------- paged / block-sparse ----
+
+def run_kv_variant(args):
+    """Decode steps over a paged cache or a block-sparse key selection. The
+    value is the KV-read bandwidth of the keys actually attended; the R = 0
+    path on the same inputs runs in alternating blocks beside it."""
+    if args.impl == "reference":
+        print(json.dumps({"impl": "reference", "unavailable":
+                          "the reference arm times the contiguous decode only"}))
+        return 0
+    from parameterized_local_linear_b200 import binding
+    dist = Dist(args.gpus)
+    dist.init_gpu()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    binding.load_library()
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.set_stream(stream)
+    w = inputs.WORKLOADS[args.workload]
+    if args.batch is not None:
+        w = inputs.Workload(w.name + f"-B{args.batch}", args.batch, w.Hq, w.Hkv, w.D, w.Lmax,
+                            w.dtype, w.seed, w.lengths, w.r_scale, w.k_offset_std, w.scale)
+    esz = 2
+    if args.kv_mode == "paged":
+        x = inputs.make_paged(w, args.page_size, dev)
+        lens = x["seqlens"].to(torch.int64).clamp(0, w.Lmax)
+        keys = int(lens.sum())
+        plan_len = x["table"].shape[1] * args.page_size
+        desc = f"paged: page_size {args.page_size}, pages scattered by a seeded permutation"
+    else:
+        x = inputs.make_block_sparse(w, args.density, dev)
+        lens = x["seqlens"].to(torch.int64).clamp(0, w.Lmax).cpu()
+        ids, cnt = x["block_ids"].cpu(), x["num_blocks"].cpu()
+        keys = 0
+        for b in range(w.B):
+            blk = ids[b, :int(cnt[b])].to(torch.int64)
+            keys += int((lens[b] - 64 * blk).clamp(0, 64).sum())
+        plan_len = 64 * x["block_ids"].shape[1]
+        desc = f"block-sparse: {args.density:.2f} of each sequence's 64-key blocks, seeded"
+    step_kv = 2 * keys * w.Hkv * w.D * esz
+    ws = binding.Workspace(w.B, w.Hq, w.Hkv, w.D, plan_len, args.num_splits, device=dev)
+    out = torch.empty((w.B, w.Hq, w.D), device=dev, dtype=torch.bfloat16)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    pool_bytes = 2 * x["k"].numel() * esz
+    # a pool smaller than the L2: rotate over enough copies of K and V to
+    # exceed twice the L2, replayed from CUDA graphs (as the contiguous bench)
+    nbuf = max(1, math.ceil(2 * l2 / pool_bytes)) if pool_bytes < 2 * l2 else 1
+    kvs = [(x["k"], x["v"])] + [(x["k"].clone(), x["v"].clone()) for _ in range(nbuf - 1)]
+
+    def step(probe, j=0):
+        kk, vv = kvs[j % nbuf]
+        if args.kv_mode == "paged":
+            binding.parallax_decode_paged(x["q"], x["r"], kk, vv, x["table"],
+                                          x["seqlens"], scale=x["scale"], out=out, workspace=ws,
+                                          num_splits=args.num_splits, probe=probe, stream=stream)
+        else:
+            binding.parallax_decode_block_sparse(x["q"], x["r"], kk, vv, x["block_ids"],
+                                                 x["num_blocks"], x["seqlens"], scale=x["scale"],
+                                                 out=out, workspace=ws, num_splits=args.num_splits,
+                                                 probe=probe, stream=stream)
+
+    graphs = {}
+    if nbuf > 1:
+        for probe in (True, False):
+            for j in range(nbuf):
+                step(probe, j)
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for j in range(nbuf):
+                    step(probe, j)
+            graphs[probe] = g
+
+    def run(k_steps, probe=True):
+        if nbuf > 1:
+            for _ in range(max(1, k_steps // nbuf)):
+                graphs[probe].replay()
+            return
+        for i in range(k_steps):
+            step(probe, i)
+
+    def timed(fn, k_steps, w_steps, sampler=None):
+        fn(w_steps)
+        torch.cuda.synchronize()
+        dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if sampler:
+            sampler.__enter__()
+        e0.record(stream)
+        fn(k_steps)
+        e1.record(stream)
+        e1.synchronize()
+        if sampler:
+            sampler.__exit__(None, None, None)
+        torch.cuda.synchronize()
+        dist.barrier()
+        return dist.max(e0.elapsed_time(e1) / 1e3)
+
+    if nbuf > 1:  # whole graph chains only
+        args.steps = max(nbuf, args.steps // nbuf * nbuf)
+    sampler = ClockSampler(dev.index)
+    t = timed(run, args.steps, args.warmup, sampler)
+    per = {True: [], False: []}
+    blk = max(1, min(args.steps, 20)) if nbuf == 1 else nbuf * max(1, 800 // nbuf)
+    for _ in range(5):
+        for probe in (True, False):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            run(blk, probe)
+            b.record(stream)
+            b.synchronize()
+            per[probe].append(a.elapsed_time(b) / 1e3 / blk)
+    t_p, t_s = dist.max(statistics.median(per[True])), dist.max(statistics.median(per[False]))
+    rc, bits = ws.status()
+    if rc != 0:
+        raise SystemExit(f"device status after timing: {binding.parallax_status_string(rc)}")
+    # end to end: q, r and lengths from pinned host memory, the output back
+    pin = {k: x[k].cpu().pin_memory() for k in ("q", "r", "seqlens")}
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+
+    def run_e2e(k_steps):
+        for i in range(k_steps):
+            for k in pin:
+                x[k].copy_(pin[k], non_blocking=True)
+            step(True, i)
+            out_host.copy_(out, non_blocking=True)
+
+    k_e2e = min(args.steps, 50)
+    t_e2e = timed(run_e2e, k_e2e, 2)
+    hbm_peak, peak_src = measured_peaks()
+    N = dist.world
+    gbs = replicas.whole_job_rate(args.steps * step_kv, t, N) / 1e9
+    clocks = sampler.summary()
+    step_bytes = step_kv + qro_bytes(x)
+    line = {
+        "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": N, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": t / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": workload_desc(w) + f"; {desc}", "global_batch": w.B * N,
+                   "seq_len": w.Lmax, "parallelism": f"replicas x{N}" if N > 1 else "single GPU",
+                   "attended_keys_per_step": keys * w.Hkv, "num_splits": args.num_splits,
+                   "l2": (f"rotate {nbuf} K/V pool copies ({nbuf * pool_bytes / 1e6:.0f} MB "
+                          f"> 2x L2), CUDA graphs" if nbuf > 1
+                          else f"pool ({pool_bytes / 1e9:.1f} GB) larger than L2")},
+        "us_per_step": t / args.steps * 1e6,
+        "kv_gbs_frac_of_hbm_peak": gbs / N / hbm_peak,
+        "softmax_r0": {"us_per_step": t_s * 1e6, "parallax_us_per_step_same_blocks": t_p * 1e6,
+                       "parallax_over_softmax_latency": t_p / t_s,
+                       "method": f"5 alternating blocks of {blk} steps each, medians"},
+        "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons", "samples")},
+        "e2e": {"value": N * k_e2e * step_kv / t_e2e / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": sum(t_.numel() * t_.element_size() for t_ in pin.values()),
+                "d2h_bytes_per_step": out_host.numel() * out_host.element_size(),
+                "us_per_step": t_e2e / k_e2e * 1e6},
+        "gpu_launches": 2 * args.steps,
+        "roofline": {"bound": "hbm", "achieved": step_bytes / (t / args.steps) / 1e9,
+                     "peak": hbm_peak, "unit": "GB/s",
+                     "frac": step_bytes / (t / args.steps) / 1e9 / hbm_peak, "traffic": None,
+                     "kernel": "whole step (split-KV + merge)", "peak_source": peak_src,
+                     "algorithmic_bytes_per_step": step_bytes},
+        "cpu_baseline": None,
+    }
+    if dist.rank == 0:
+        print(json.dumps(line))
+    dist.close()
+    return 0
+
+
 # ------------------------------------------------------------- GPU timing ----
 
 def main():
     args = parse_args()
     if args.prefill:
         return run_prefill(args)
+    if args.kv_mode != "contiguous":
+        return run_kv_variant(args)
     if args.impl == "reference":
         return run_reference(args)
 

@@ -146,3 +146,49 @@ def custom_workload(name: str, B: int, Hq: int, Hkv: int, D: int, Lmax: int,
         lengths = tuple(int(x) for x in lengths)
     return Workload(name, B, Hq, Hkv, D, Lmax, dtype, seed, lengths, r_scale,
                     k_offset_std, scale)
+
+
+def make_paged(w: Workload, page_size: int, device="cpu") -> dict:
+    """Workload `w` with its cache in pages: a pool [B * ceil(Lmax / page_size),
+    page_size, Hkv, D] of N(0,1) keys and values (the workload's key offsets
+    are not applied) and a block table that scatters each sequence's pages
+    through the pool in a seeded random order."""
+    device = torch.device(device)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(w.seed)
+    dt = w.dtype
+    q = torch.randn((w.B, w.Hq, w.D), generator=gen, device=device, dtype=dt)
+    r = torch.randn((w.B, w.Hq, w.D), generator=gen, device=device, dtype=dt)
+    if w.r_scale != 1.0:
+        r = (r * w.r_scale).to(dt)
+    per = (w.Lmax + page_size - 1) // page_size
+    pool = (w.B * per, page_size, w.Hkv, w.D)
+    k = torch.randn(pool, generator=gen, device=device, dtype=dt)
+    v = torch.randn(pool, generator=gen, device=device, dtype=dt)
+    seqlens = draw_lengths(w, gen, device)
+    perm = torch.randperm(w.B * per, generator=gen, device=device)
+    table = perm.reshape(w.B, per).to(torch.int32)
+    return {"q": q, "r": r, "k": k, "v": v, "seqlens": seqlens, "table": table,
+            "page_size": page_size, "scale": w.qk_scale}
+
+
+def make_block_sparse(w: Workload, density: float, device="cpu") -> dict:
+    """Workload `w` (dense cache, padding left as drawn) plus, per sequence, a
+    seeded random subset of about `density` of the 64-key blocks below its
+    length (at least one), sorted, padded to the longest list."""
+    x = make_inputs(w, device=device, pad_value=None)
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(w.seed + 1000)
+    lens = x["seqlens"].cpu().tolist()
+    lists = []
+    for n in lens:
+        nb = max(1, (int(n) + 63) // 64)
+        take = max(1, int(round(density * nb)))
+        lists.append(torch.sort(torch.randperm(nb, generator=gen)[:take]).values)
+    width = max(len(a) for a in lists)
+    ids = torch.zeros((w.B, width), dtype=torch.int32)
+    for b, a in enumerate(lists):
+        ids[b, :len(a)] = a.to(torch.int32)
+    x["block_ids"] = ids.to(device)
+    x["num_blocks"] = torch.tensor([len(a) for a in lists], dtype=torch.int32, device=device)
+    return x
