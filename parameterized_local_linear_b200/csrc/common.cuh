@@ -39,20 +39,26 @@ struct DecodeParams {
 
 // ------------------------------------------------ TMA kernel geometry ------
 constexpr int kTileKeys = 64;        // keys per pipeline stage
-constexpr int kConsumerWarps = 4;    // each owns 16 keys of a stage
-constexpr int kTcThreads = (kConsumerWarps + 1) * 32;  // + one producer warp
+constexpr int kConsumerWarps = 4;    // warps per stage: each owns 16 of its keys
+constexpr int kConsumerGroups = 2;   // groups of kConsumerWarps that take alternate stages
+constexpr int kTcConsumers = kConsumerWarps * kConsumerGroups;
+constexpr int kTcThreads = (kTcConsumers + 1) * 32;  // + one producer warp
 constexpr int kBoxBytes = kTileKeys * 128;             // one 64-key x 128-byte swizzled box
 
-// A 96 KB ring of K+V per CTA: measured on B200, one CTA per SM with 96 KB
-// in flight streams faster than 192 KB per SM (one CTA with a 6-stage ring,
-// or two CTAs), and it leaves shared memory for the merge kernel's blocks to
-// become resident early.
+// A 96-128 KB ring of K+V per CTA: measured on B200, one CTA per SM with
+// ~100 KB in flight streams faster than 192 KB per SM (one CTA with a 6-stage
+// ring, or two CTAs), and it leaves shared memory for the merge kernel's blocks
+// to become resident early. The stage count is a multiple of the consumer
+// groups, so every stage is always consumed by the same group: a group then
+// waits on each of its stages' fills in order, never two phases ahead of an
+// mbarrier (where a parity wait can not tell the fills apart).
 template <int D>
 struct TcGeom {
   static constexpr int kHalves = D / 64;                 // 128-byte boxes per key row
   static constexpr int kKBytes = kHalves * kBoxBytes;    // K tile of one stage
   static constexpr int kStageBytes = 2 * kKBytes;        // K + V
-  static constexpr int kStages = D == 128 ? 3 : 6;
+  static constexpr int kStages = D == 128 ? 4 : 6;
+  static_assert(kStages % kConsumerGroups == 0, "a stage must always belong to one group");
 };
 
 __host__ __device__ constexpr int align_up(int x, int a) { return (x + a - 1) / a * a; }
@@ -67,8 +73,8 @@ __host__ __device__ inline TcSmemLayout tc_smem_layout(int D, int stage_bytes, i
   (void)probe;
   TcSmemLayout L{};
   L.off_p = stages * stage_bytes;
-  L.off_merge = L.off_p + kConsumerWarps * 512;
-  L.off_bar = align_up(L.off_merge + kConsumerWarps * G * rec_floats(D) * 4, 16);
+  L.off_merge = L.off_p + kTcConsumers * 512;
+  L.off_bar = align_up(L.off_merge + kTcConsumers * G * rec_floats(D) * 4, 16);
   // full[stages], empty[stages], fin[2]
   L.off_misc = L.off_bar + 8 * (2 * stages + 2);
   L.total = L.off_misc + 48 + 1024;  // abort flag, per-stage valid keys, alignment slack

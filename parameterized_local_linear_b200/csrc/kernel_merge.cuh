@@ -90,18 +90,17 @@ __global__ void __launch_bounds__(kMergeThreads, 4) parallax_merge_kernel(const 
   for (int j0 = 0; j0 < S; j0 += chunk) {
     const int nch = min(chunk, S - j0);
     float m = kNegInf, l = 0.f, bb = 0.f;
-    if (tid < nch * G) {
-      const float* rec = record(j0 + tid / G, tid % G);
-      m = rec[0];
-      l = rec[1];
-      bb = PROBE ? rec[2] : 0.f;
+    if (tid < nch * G) {  // the record header (m, l, b, -) in one load
+      const float4 hd = ld_cg_f4(record(j0 + tid / G, tid % G));
+      m = hd.x;
+      l = hd.y;
+      bb = PROBE ? hd.z : 0.f;
     }
     float4 v[kMergeChunk];
 #pragma unroll
     for (int k = 0; k < kMergeChunk; ++k)
-      v[k] = (active && k < nch)
-                 ? *reinterpret_cast<const float4*>(record(j0 + k, h_col) + kRecHead + ac * D + 4 * d4)
-                 : make_float4(0.f, 0.f, 0.f, 0.f);
+      v[k] = (active && k < nch) ? ld_cg_f4(record(j0 + k, h_col) + kRecHead + ac * D + 4 * d4)
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
     if (tid < nch * G) {
       s_m[tid] = m;
       s_l[tid] = l;

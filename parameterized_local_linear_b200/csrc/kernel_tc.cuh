@@ -5,9 +5,11 @@
 // streams 64-key K and V tiles of the current item with one TMA each (5-D
 // tensor maps {64 dims, keys, D/64 halves, kv heads, batch rows} over either
 // cache layout, 128-byte swizzle, no multicast) into a ring of shared-memory
-// stages guarded by full/empty mbarriers. Warps 0..3 consume: warp w owns keys 16w..16w+15 of every stage
-// and keeps its own online accumulators, so the consumer warps never
-// synchronise inside the key loop. They read the q (and r) rows of the item's
+// stages guarded by full/empty mbarriers. Warp 8 is the producer; warps 0..7
+// consume in two groups of four that take alternate stages (two tiles in
+// flight through the math at once): warp w owns keys 16 (w % 4) .. +15 of its
+// group's stages and keeps its own online accumulators, so the consumer warps
+// never synchronise inside the key loop. They read the q (and r) rows of the item's
 // GQA group straight into mma fragments from global memory, overlapped with
 // the first K/V tile's flight.
 //
@@ -30,7 +32,7 @@
 // result itself can be ~0 (one dominant key); l and b are summed from the same
 // hi + lo values the tensor cores apply. The softmax kernel splits only for
 // the fp32-output mode.
-// At the end of a piece the four warps combine their (m, l, b, A, C) in shared
+// At the end of a piece the eight warps combine their (m, l, b, A, C) in shared
 // memory; a whole item is finished (o = A/l + C/l - (b/l)(A/l), or A/l without
 // the probe) and stored, a partial item writes a partial record for the merge
 // kernel.
@@ -97,12 +99,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(bar_full + 8 * s, 1);
       mbar_init(bar_empty + 8 * s, kConsumerWarps);
     }
-    for (int s = 0; s < 2; ++s) mbar_init(bar_fin + 8 * s, kConsumerWarps);
+    for (int s = 0; s < 2; ++s) mbar_init(bar_fin + 8 * s, kTcConsumers);
     *abort_flag = 0;
     mbar_fence_init();
   }
   uint64_t policy = 0;
-  if (tid == kConsumerWarps * 32) {  // the producer lane: descriptors are kernel parameters
+  if (tid == kTcConsumers * 32) {  // the producer lane: descriptors are kernel parameters
     prefetch_tensormap(&tmK);
     prefetch_tensormap(&tmV);
     policy = l2_policy_evict_first();
@@ -123,7 +125,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int G = p.G;
 
   // ------------------------------------------------------------ producer --
-  if (warp == kConsumerWarps) {
+  if (warp == kTcConsumers) {
     if (lane != 0) return;
     PieceCursor cur;
     cur.init(part, key_space(p), p.B, p.Hkv);
@@ -177,7 +179,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   // ----------------------------------------------------------- consumers --
   const int g8 = lane >> 2, c4 = lane & 3;
-  const int my0 = 16 * warp;  // this warp's first key row inside a stage
+  const int group = warp / kConsumerWarps;  // takes the stages of tiles group, group + 2, ...
+  const int my0 = 16 * (warp % kConsumerWarps);  // this warp's first key row inside a stage
   const uint32_t p_tile = base + L.off_p + warp * 512;
   float* const merge_scr = reinterpret_cast<float*>(gbase + L.off_merge);
   const int REC = rec_floats(D);
@@ -195,7 +198,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   cur.init(part, key_space(p), p.B, p.Hkv);
   Piece pc;
   int stage = 0;
-  uint32_t ph = 0, fph = 0;
+  uint32_t ph = 0, fph = 0, tseq = 0;  // tseq: the CTA's tile count, all pieces
   bool ok = true, triggered = false;
 
   while (ok && cur.next(pc)) {
@@ -229,7 +232,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     float m0 = kNegInf, m1 = kNegInf, l0 = 0.f, l1 = 0.f;  // (m1, l1) softmax only
     float bsum = 0.f;                                     // PROBE only
 
-    for (int k0 = pc.i; k0 < pc.i + pc.len; k0 += kTileKeys) {
+    for (int k0 = pc.i; k0 < pc.i + pc.len; k0 += kTileKeys, ++tseq) {
+      if ((int)(tseq % kConsumerGroups) != group) {  // the other group's tile
+        if (++stage == kStages) {
+          stage = 0;
+          ph ^= 1;
+        }
+        continue;
+      }
       if (!mbar_wait_bounded(bar_full + 8 * stage, ph, p.timeout_ns, abort_flag)) {
         ok = false;
         break;
@@ -453,14 +463,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     {
       const int ctid = tid;  // 0..127
-      for (int idx = ctid; idx < G * D; idx += kConsumerWarps * 32) {
+      for (int idx = ctid; idx < G * D; idx += kTcConsumers * 32) {
         const int h = idx / D, d = idx - h * D;
         float M = kNegInf;
 #pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, merge_scr[(w * G + h) * REC]);
+        for (int w = 0; w < kTcConsumers; ++w) M = fmaxf(M, merge_scr[(w * G + h) * REC]);
         float Lw = 0.f, Bw = 0.f, Aw = 0.f, Cw = 0.f;
 #pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) {
+        for (int w = 0; w < kTcConsumers; ++w) {
           const float* rec = merge_scr + (w * G + h) * REC;
           const float mw = rec[0];
           const float a = mw == kNegInf ? 0.f : ex2_approx(mw - M);

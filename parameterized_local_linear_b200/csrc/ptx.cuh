@@ -192,6 +192,15 @@ __device__ __forceinline__ float bf16_hi_to_float(uint32_t v) {
 
 // ------------------------------------------- programmatic dependent launch --
 
+// 16-byte global load cached in L2 only (data another CTA wrote moments ago).
+__device__ __forceinline__ float4 ld_cg_f4(const void* p) {
+  float4 v;
+  asm volatile("ld.global.cg.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "l"(p));
+  return v;
+}
+
 __device__ __forceinline__ void pdl_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
