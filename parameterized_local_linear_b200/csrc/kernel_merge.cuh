@@ -96,11 +96,13 @@ __global__ void __launch_bounds__(kMergeThreads, 4) parallax_merge_kernel(const 
       l = hd.y;
       bb = PROBE ? hd.z : 0.f;
     }
+    // every thread loads kMergeChunk records unconditionally (past the chunk it
+    // re-reads the chunk's last record, weighted 0 below), so the loads issue
+    // back to back with no branch between them
     float4 v[kMergeChunk];
 #pragma unroll
     for (int k = 0; k < kMergeChunk; ++k)
-      v[k] = (active && k < nch) ? ld_cg_f4(record(j0 + k, h_col) + kRecHead + ac * D + 4 * d4)
-                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+      v[k] = ld_cg_f4(record(j0 + min(k, nch - 1), h_col) + kRecHead + ac * D + 4 * d4);
     if (tid < nch * G) {
       s_m[tid] = m;
       s_l[tid] = l;
