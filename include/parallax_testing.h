@@ -1,9 +1,9 @@
 /*
  * parallax_testing.h - testing hook of libparallax.so.
  *
- * Not part of the decode API, and with no counterpart in the pages: it exists
- * so that tests can watch the kernels' bounded waits give up on a GPU without
- * hanging or faulting it.
+ * Not part of the API, and with no counterpart in the pages: these hooks
+ * exist so that tests can watch the kernels' bounded waits give up on a GPU
+ * without hanging or faulting it.
  */
 #ifndef PARALLAX_TESTING_H
 #define PARALLAX_TESTING_H
@@ -29,6 +29,19 @@ int parallax_testing_decode_stalled(const void* q, const void* r, const void* k_
                                     void* out, int B, int Hq, int Hkv, int D, float scale,
                                     void* stream, int Lmax, int num_splits, void* workspace,
                                     size_t workspace_bytes, int timeout_ms);
+
+/*
+ * parallax_prefill (same arguments and checks) with the same two changes for
+ * the tcgen05 forward: every wait bounded by timeout_ms (1 .. 10000), and the
+ * TMA producer never loads the first K tile of each CTA, so the UMMA issuer's
+ * wait on it runs out. Each CTA then records PARALLAX_DEVICE_STATUS_TIMEOUT,
+ * waits (bounded) for its own copies in flight, frees its tensor memory and
+ * returns; the output is invalid; the CUDA context stays usable.
+ */
+int parallax_testing_prefill_stalled(const void* q, const void* r, const void* k, const void* v,
+                                     void* out, int B, int Hq, int Hkv, int L, int D,
+                                     float scale, int causal, void* stream, int out_dtype,
+                                     void* workspace, size_t workspace_bytes, int timeout_ms);
 
 #ifdef __cplusplus
 }

@@ -55,6 +55,7 @@ struct PrefillParams {
   int total;                // packed layout: rows of q, k (cu_seqlens is clamped to it)
   float scale_log2;         // > 0
   unsigned long long timeout_ns;
+  int debug_skip_first_k;   // testing hook: the producer never loads the first K tile
 };
 
 template <int D>
@@ -171,6 +172,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     // ------------------------------------------------------------ producer --
     if (lane == 0) {
       bool ok = true;
+      bool skipped_k0 = false;  // testing hook
       int last = -1;  // the last tile whose K and V loads were both started
       mbar_arrive_expect_tx(bar_q, 2 * Geo::kQBytes);
       tma_load_4d(sQ, &tmQ, 0, qrow, 0, qitem, bar_q, policy);
@@ -182,11 +184,16 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           ok = false;
           break;
         }
-        mbar_arrive_expect_tx(k_full + 8 * st, Geo::kKVBytes);
-        tma_load_4d(sK + st * Geo::kKVBytes, &tmK, 0, krow + j * kPfKeys, 0, kitem,
-                    k_full + 8 * st, policy);
+        if (j == 0 && p.debug_skip_first_k) {
+          skipped_k0 = true;  // the UMMA issuer's wait on this tile must run out
+        } else {
+          mbar_arrive_expect_tx(k_full + 8 * st, Geo::kKVBytes);
+          tma_load_4d(sK + st * Geo::kKVBytes, &tmK, 0, krow + j * kPfKeys, 0, kitem,
+                      k_full + 8 * st, policy);
+        }
         if (!mbar_wait_bounded(v_empty + 8 * st, ph ^ 1, p.timeout_ns, abort_flag)) {
-          mbar_wait_bounded(k_full + 8 * st, ph, p.timeout_ns, nullptr);  // K_j in flight
+          if (!skipped_k0 || j > 0)
+            mbar_wait_bounded(k_full + 8 * st, ph, p.timeout_ns, nullptr);  // K_j in flight
           ok = false;
           break;
         }
@@ -209,7 +216,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       for (int j = max(0, last - kPfStages + 1); j <= last; ++j) {
         const int s = j % kPfStages;
         const uint32_t par = (uint32_t)(j / kPfStages) & 1u;
-        mbar_wait_bounded(k_full + 8 * s, par, p.timeout_ns, nullptr);
+        if (!(j == 0 && skipped_k0)) mbar_wait_bounded(k_full + 8 * s, par, p.timeout_ns, nullptr);
         mbar_wait_bounded(v_full + 8 * s, par, p.timeout_ns, nullptr);
       }
     }

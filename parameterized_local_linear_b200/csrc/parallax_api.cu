@@ -593,10 +593,12 @@ int check_prefill_args(const void* q, const void* r, const void* k, const void* 
 
 }  // namespace
 
-extern "C" int parallax_prefill(const void* q, const void* r, const void* k, const void* v,
-                                void* out, int B, int Hq, int Hkv, int L, int D, float scale,
-                                int causal, void* stream, int out_dtype, void* workspace,
-                                size_t workspace_bytes) {
+namespace {
+
+int run_prefill(const void* q, const void* r, const void* k, const void* v, void* out, int B,
+                int Hq, int Hkv, int L, int D, float scale, int causal, void* stream,
+                int out_dtype, void* workspace, size_t workspace_bytes,
+                unsigned long long timeout_ns, int debug_skip_first_k) {
   int st = check_prefill_args(q, r, k, v, out, Hq, Hkv, D, scale, out_dtype, workspace,
                               workspace_bytes);
   if (st != PARALLAX_OK) return st;
@@ -612,9 +614,30 @@ extern "C" int parallax_prefill(const void* q, const void* r, const void* k, con
   prm.num_qt = (L + kPfRows - 1) / kPfRows;
   prm.causal = causal != 0;
   prm.scale_log2 = (float)((double)scale * 1.4426950408889634);
-  prm.timeout_ns = kDefaultTimeoutNs;
+  prm.timeout_ns = timeout_ns;
+  prm.debug_skip_first_k = debug_skip_first_k;
   return dispatch_prefill<false>(q, r, k, v, prm, D, out_dtype == PARALLAX_DTYPE_F32,
                                  prm.num_qt, static_cast<cudaStream_t>(stream));
+}
+
+}  // namespace
+
+extern "C" int parallax_prefill(const void* q, const void* r, const void* k, const void* v,
+                                void* out, int B, int Hq, int Hkv, int L, int D, float scale,
+                                int causal, void* stream, int out_dtype, void* workspace,
+                                size_t workspace_bytes) {
+  return run_prefill(q, r, k, v, out, B, Hq, Hkv, L, D, scale, causal, stream, out_dtype,
+                     workspace, workspace_bytes, kDefaultTimeoutNs, 0);
+}
+
+extern "C" int parallax_testing_prefill_stalled(const void* q, const void* r, const void* k,
+                                                const void* v, void* out, int B, int Hq,
+                                                int Hkv, int L, int D, float scale, int causal,
+                                                void* stream, int out_dtype, void* workspace,
+                                                size_t workspace_bytes, int timeout_ms) {
+  if (timeout_ms < 1 || timeout_ms > 10000) return PARALLAX_ERR_BAD_SHAPE;
+  return run_prefill(q, r, k, v, out, B, Hq, Hkv, L, D, scale, causal, stream, out_dtype,
+                     workspace, workspace_bytes, (unsigned long long)timeout_ms * 1000000ull, 1);
 }
 
 extern "C" int parallax_varlen_prefill(const void* q, const void* r, const void* k,

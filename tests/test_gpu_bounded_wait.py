@@ -49,3 +49,41 @@ def test_bounded_wait_gives_up_and_context_survives():
     assert np.all(np.isfinite(g))
     assert np.max(np.abs(g - ref) / np.maximum(1.0, np.abs(ref))) <= 1e-4
     assert ws.status() == (0, 0)
+
+
+def test_prefill_bounded_wait_gives_up_and_context_survives():
+    """The tcgen05 prefill: the producer never loads a CTA's first K tile, so
+    the UMMA issuer's wait runs out (50 ms); every CTA must record the timeout,
+    drain its own copies, free its tensor memory and return, and a normal
+    prefill on the same context (which allocates tensor memory again on every
+    SM) must then match the oracle."""
+    lib = binding.load_library()
+    fn = lib.parallax_testing_prefill_stalled
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    fn.argtypes = [vp] * 5 + [i] * 5 + [ctypes.c_float, i, vp, i, vp, ctypes.c_size_t, i]
+    fn.restype = i
+    B, Hq, Hkv, L, D = 2, 4, 2, 300, 128
+    g = torch.Generator(device="cuda").manual_seed(33)
+    mk = lambda H, sc=1.0: (torch.randn(B, H, L, D, device="cuda", generator=g) * sc).to(
+        torch.bfloat16)
+    q, r, k, v = mk(Hq), mk(Hq, 0.5), mk(Hkv), mk(Hkv)
+    out = torch.empty_like(q)
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream().cuda_stream
+    t0 = time.perf_counter()
+    rc = fn(q.data_ptr(), r.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, Hq, Hkv, L,
+            D, D ** -0.5, 1, stream, 0, ws.data_ptr(), ws.numel(), 50)
+    assert rc == 0
+    torch.cuda.synchronize()
+    elapsed = time.perf_counter() - t0
+    bits = int(ws[:4].view(torch.int32).item())
+    assert bits & TIMEOUT_BIT, bits
+    assert elapsed < 5.0, f"the stalled call took {elapsed:.2f} s"
+    ws.zero_()
+    got = binding.parallax_prefill(q, r, k, v, out_dtype=torch.float32, workspace=ws)
+    want = oracle.parallax_prefill(q, r, k, v, D ** -0.5, True)
+    gg = got.double().cpu().numpy()
+    assert np.all(np.isfinite(gg))
+    assert np.max(np.abs(gg - want) / np.maximum(1.0, np.abs(want))) <= 1e-4
+    torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32).item()) == 0
