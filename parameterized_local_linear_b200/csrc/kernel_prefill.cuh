@@ -28,8 +28,8 @@
 //           with the weights the products apply. O is rescaled in TMEM only
 //           when the max grows by more than 2^8 (otherwise the stale max keeps
 //           every e <= 2^8); each thread of a row rescales one of O_A, O_C.
-// TMEM columns: S [0,64) T [64,128) P [128,256) (P_hi, P_lo, PT_hi, PT_lo,
-// 32 columns each), O_A [256, 256+D), O_C [256+D, 256+2D).
+// TMEM columns: S [0,64) T [64,128) P [128,256) (per key half, 64 columns:
+// P_hi, P_lo, PT_hi, PT_lo, 16 each), O_A [256, 256+D), O_C [256+D, 256+2D).
 // Every wait is bounded; on a timeout the kernel records it, waits (bounded)
 // for its own TMA copies and UMMAs in flight, frees TMEM and returns.
 #pragma once
@@ -269,7 +269,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 #pragma unroll
             for (int kk = 0; kk < kPfKeys / 16; ++kk) {
               const bool acc = !(j == 0 && (pm & 1) == 0 && kk == 0);
-              umma_bf16_ts(dO, tmem + kPfColP + 32 * pm + 8 * kk,
+              // keys 16 kk .. +15 sit in half kk / 2's 64 columns: 16 per operand
+              umma_bf16_ts(dO, tmem + kPfColP + 64 * (kk >> 1) + 16 * pm + 8 * (kk & 1),
                            umma_smem_desc(sVs + kk * 16 * 128, kPfKeys * 128, 1024), kIdescPV,
                            acc);
             }
@@ -291,7 +292,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const int r = quarter * 32 + lane, qi = q0 + r;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const uint32_t tS = tmem + lane_base + kPfColS, tT = tmem + lane_base + kPfColT;
-    const uint32_t tP = tmem + lane_base + kPfColP + 16 * half;  // this half's 16 columns
+    const uint32_t tP = tmem + lane_base + kPfColP + 64 * half;  // this half's 64 columns
     const float c = p.scale_log2;
     float m_used = kNegInf, l = 0.f, bsum = 0.f;
     bool ok = true;
@@ -336,8 +337,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         m_used = mx;
       }
       const float neg_m = -m_used;
-      // e and e*s of this thread's 32 keys as exact bf16 hi + lo pairs
-      uint32_t ph[16], pl[16], th[16], tl[16];
+      // e and e*s of this thread's 32 keys as exact bf16 hi + lo pairs, in the
+      // order of this half's P columns: P_hi | P_lo then PT_hi | PT_lo
+      uint32_t pp[32], pt[32];
+      uint32_t* const ph = pp;
+      uint32_t* const pl = pp + 16;
+      uint32_t* const th = pt;
+      uint32_t* const tl = pt + 16;
       float lt = 0.f, bt = 0.f;
 #pragma unroll
       for (int u = 0; u < 16; ++u) {
@@ -373,10 +379,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       }
       l = l * alpha + lt;
       bsum = bsum * alpha + bt;
-      tmem_st16(tP + 0 * 32, ph);
-      tmem_st16(tP + 1 * 32, pl);
-      tmem_st16(tP + 2 * 32, th);
-      tmem_st16(tP + 3 * 32, tl);
+      tmem_st32u(tP, pp);
+      tmem_st32u(tP + 32, pt);
       tmem_wait_st();
       tc_fence_before_sync();
       __syncwarp();
