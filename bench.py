@@ -660,6 +660,11 @@ def run_kv_variant(args):
 
     k_e2e = min(args.steps, 50)
     t_e2e = timed(run_e2e, k_e2e, 2)
+    # CPU baseline: the oracle (it gathers the same keys into a dense cache) on
+    # the first batch rows, as many as fit in the budget (rank 0, N = 1 only)
+    cpu = None
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        cpu = kv_variant_oracle_sample(args, w, x, min(10.0, args.cpu_seconds))
     hbm_peak, peak_src = measured_peaks()
     N = dist.world
     gbs = replicas.whole_job_rate(args.steps * step_kv, t, N) / 1e9
@@ -691,12 +696,55 @@ def run_kv_variant(args):
                      "frac": step_bytes / (t / args.steps) / 1e9 / hbm_peak, "traffic": None,
                      "kernel": "whole step (split-KV + merge)", "peak_source": peak_src,
                      "algorithmic_bytes_per_step": step_bytes},
-        "cpu_baseline": None,
+        "cpu_baseline": cpu,
     }
     if dist.rank == 0:
         print(json.dumps(line))
     dist.close()
     return 0
+
+
+def kv_variant_oracle_sample(args, w, x, budget_s):
+    """The fp64 oracle on the first batch rows of a paged or block-sparse
+    step: time one row, then as many rows as fit in budget_s. GB/s of the K/V
+    the rows attend."""
+    import oracle
+    scale, esz = x["scale"], 2
+
+    def rows_input(n_rows):
+        idx = slice(0, n_rows)
+        q, r, lens = x["q"][idx].cpu(), x["r"][idx].cpu(), x["seqlens"][idx].cpu()
+        if args.kv_mode == "paged":
+            table = x["table"][idx].cpu()
+            used = torch.unique(table)  # only the pages these rows use, renumbered
+            remap = torch.full((int(used.max()) + 1,), -1, dtype=torch.int64)
+            remap[used] = torch.arange(used.numel())
+            dev_used = used.to(x["k"].device)
+            kp, vp = x["k"][dev_used].cpu(), x["v"][dev_used].cpu()
+            keys = int(lens.to(torch.int64).clamp(0, w.Lmax).sum())
+            call = lambda: oracle.parallax_decode_paged(q, r, kp, vp, remap[table.long()].numpy(),
+                                                        lens, scale)
+        else:
+            ids, cnt = x["block_ids"][idx].cpu(), x["num_blocks"][idx].cpu()
+            k, v = x["k"][idx].cpu(), x["v"][idx].cpu()
+            keys = sum(int((lens[b].long() - 64 * ids[b, :int(cnt[b])].long()).clamp(0, 64).sum())
+                       for b in range(n_rows))
+            call = lambda: oracle.parallax_decode_block_sparse(q, r, k, v, ids, cnt, lens, scale)
+        return call, 2 * keys * w.Hkv * w.D * esz
+
+    call, _ = rows_input(1)
+    t0 = time.perf_counter()
+    call()
+    one = max(1e-3, time.perf_counter() - t0)
+    n_rows = max(1, min(w.B, int(budget_s / one), 16))
+    call, kv = rows_input(n_rows)
+    t0 = time.perf_counter()
+    call()
+    secs = time.perf_counter() - t0
+    return {"value": kv / secs / 1e9, "unit": "GB/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"fp64 oracle ({args.kv_mode}: the same keys gathered into a dense cache), "
+                      f"one pass over batch rows 0..{n_rows - 1} ({n_rows} of {w.B}); {secs:.1f} s"}
 
 
 # ------------------------------------------------------------- GPU timing ----
