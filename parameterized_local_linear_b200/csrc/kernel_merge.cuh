@@ -67,7 +67,7 @@ __global__ void __launch_bounds__(kMergeThreads, 4) parallax_merge_kernel(const 
   if ((long long)(part.n - part.i) > part.hi - part.lo) return;  // it ends in a later partition
 
   const long long s0 = part.lo - part.i;  // item start
-  const int c_lo = (int)(s0 / part.per);
+  const int c_lo = (int)div_pos(s0, part.per);
   const int S = c - c_lo + 1;  // pieces of the item, in partition order
   const int D = p.D, G = p.G, REC = rec_floats(D), D4 = D / 4;
   const bool lo_is_first = s0 == (long long)c_lo * part.per;

@@ -502,6 +502,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
       }
     }
+    if (cur.pos >= cur.hi) break;  // the CTA's last piece: no one overwrites the scratch
     __syncwarp();  // scratch may be overwritten by the next piece
     if (lane == 0) mbar_arrive(bar_fin + 8);
     if (!mbar_wait_bounded(bar_fin + 8, fph, p.timeout_ns, abort_flag)) {

@@ -19,6 +19,13 @@ namespace plx {
 
 constexpr int kRangeAlign = 64;  // partition ranges are multiples of one K/V tile
 
+// x / d for x >= 0, d > 0: one 32-bit division when x fits (the usual case;
+// a 64-bit division is a long software sequence on the critical path).
+__device__ __forceinline__ long long div_pos(long long x, long long d) {
+  if (x <= 0x7fffffffLL && d <= 0x7fffffffLL) return (long long)((unsigned)x / (unsigned)d);
+  return x / d;
+}
+
 __device__ __forceinline__ int clamp_len(int n, int Lmax) {
   return n < 0 ? 0 : (n > Lmax ? Lmax : n);
 }
@@ -113,7 +120,7 @@ __device__ inline PartitionInfo locate_partition(const KeySpace& ks, int B, int 
   p.total = (long long)Hkv * __shfl_sync(0xffffffffu, incl, 31);
   // ranges are whole 64-key tiles, so a range starts on a tile of its item
   // whenever the items are tile multiples (trailing partitions may be empty)
-  p.per = ((p.total + P - 1) / P + kRangeAlign - 1) / kRangeAlign * kRangeAlign;
+  p.per = (div_pos(p.total + P - 1, P) + kRangeAlign - 1) / kRangeAlign * kRangeAlign;
   p.lo = min(p.total, (long long)c * p.per);
   p.hi = min(p.total, p.lo + p.per);
   p.b = -1;
