@@ -134,3 +134,52 @@ def test_block_sparse_bad_ids_are_flagged():
     want = oracle.parallax_decode_block_sparse(q, r, k, v, np.array([[0, 2, 0], [1, 2, 3]]),
                                                np.array([2, 3]), n, D ** -0.5)
     assert scaled_error(got, want) <= 1e-4
+
+
+@pytest.mark.parametrize("mode", ["paged", "block_sparse"])
+def test_full_size_sampled(mode):
+    """The bench's paged (large workload, page 256) and block-sparse (long
+    workload, half the blocks) steps at full size, in the bench's launch
+    configuration: two batch rows against the oracle (gathering only their
+    keys), every output finite."""
+    from parameterized_local_linear_b200 import inputs
+    if mode == "paged":
+        w = inputs.WORKLOADS["large"]
+        x = inputs.make_paged(w, 256, "cuda")
+        plan = x["table"].shape[1] * 256
+    else:
+        w = inputs.WORKLOADS["long"]
+        x = inputs.make_block_sparse(w, 0.5, "cuda")
+        plan = 64 * x["block_ids"].shape[1]
+    try:
+        ws = binding.Workspace(w.B, w.Hq, w.Hkv, w.D, plan)
+        if mode == "paged":
+            got = binding.parallax_decode_paged(x["q"], x["r"], x["k"], x["v"], x["table"],
+                                                x["seqlens"], scale=x["scale"],
+                                                out_dtype=torch.float32, workspace=ws)
+        else:
+            got = binding.parallax_decode_block_sparse(x["q"], x["r"], x["k"], x["v"],
+                                                       x["block_ids"], x["num_blocks"],
+                                                       x["seqlens"], scale=x["scale"],
+                                                       out_dtype=torch.float32, workspace=ws)
+        assert bool(torch.isfinite(got).all())
+        assert status_bits(ws) == 0
+        for b in (0, w.B - 1):
+            sl = slice(b, b + 1)
+            if mode == "paged":
+                table = x["table"][sl].cpu()
+                used = torch.unique(table)
+                remap = torch.full((int(used.max()) + 1,), -1, dtype=torch.int64)
+                remap[used] = torch.arange(used.numel())
+                dev_used = used.cuda()
+                want = oracle.parallax_decode_paged(x["q"][sl], x["r"][sl], x["k"][dev_used],
+                                                    x["v"][dev_used], remap[table.long()].numpy(),
+                                                    x["seqlens"][sl], x["scale"])
+            else:
+                want = oracle.parallax_decode_block_sparse(
+                    x["q"][sl], x["r"][sl], x["k"][sl], x["v"][sl], x["block_ids"][sl],
+                    x["num_blocks"][sl], x["seqlens"][sl], x["scale"])
+            assert scaled_error(got[sl], want) <= TOL[torch.float32], (mode, b)
+    finally:
+        del x
+        torch.cuda.empty_cache()

@@ -56,3 +56,20 @@ def test_prefill_r_zero_and_deterministic():
     b = binding.parallax_prefill(q, z, k, v, out_dtype=torch.float32)
     assert torch.equal(a, b)
     assert scaled_error(a, want) <= 1e-4
+
+
+def test_prefill_full_size_sampled():
+    """The bench's prefill workload (Qwen-3 attention heads at the training
+    length: B=4, Hq=16, Hkv=8, L=4096, D=128, the README's N(0,1) recipe with r
+    scaled by 0.5): two (batch, head) slices against the oracle, every output
+    finite."""
+    B, Hq, Hkv, L, D = 4, 16, 8, 4096, 128
+    q, r, k, v = make(B, Hq, Hkv, L, D, seed=7)
+    got = binding.parallax_prefill(q, r, k, v, out_dtype=torch.float32)
+    assert bool(torch.isfinite(got).all())
+    for b, h in ((0, 0), (3, 15)):
+        g = h // (Hq // Hkv)
+        sl = lambda t, i: t[b:b + 1, i:i + 1]
+        want = oracle.parallax_prefill(sl(q, h), sl(r, h), sl(k, g), sl(v, g), D ** -0.5, True)
+        err = scaled_error(got[b:b + 1, h:h + 1], want)
+        assert err <= TOL[torch.float32], (b, h, err)

@@ -90,3 +90,23 @@ def test_varlen_malformed_lengths_are_clamped():
     assert status_bits(ws) & 2
     binding.parallax_varlen_prefill(q, r, k, v, cu, 200, workspace=ws)
     assert status_bits(ws) == 0
+
+
+def test_varlen_full_size_sampled():
+    """The bench's varlen workload (16 sequences of lengths U{1..4096}, Hq=16,
+    Hkv=8, D=128): the shortest and the longest sequence, one head each,
+    against the oracle."""
+    lens = torch.randint(1, 4097, (16,), generator=torch.Generator().manual_seed(11)).tolist()
+    q, r, k, v, cu = make(lens, 16, 8, 128, seed=430)
+    got = binding.parallax_varlen_prefill(q, r, k, v, cu, max(lens), out_dtype=torch.float32)
+    assert bool(torch.isfinite(got).all())
+    cuh = cu.cpu().tolist()
+    for s in (int(np.argmin(lens)), int(np.argmax(lens))):
+        a, e = cuh[s], cuh[s + 1]
+        for h in (0, 13):
+            g = h // 2
+            want = oracle.parallax_varlen_prefill(q[a:e, h:h + 1], r[a:e, h:h + 1],
+                                                  k[a:e, g:g + 1], v[a:e, g:g + 1],
+                                                  np.array([0, e - a]), 128 ** -0.5)
+            err = scaled_error(got[a:e, h:h + 1], want)
+            assert err <= TOL[torch.float32], (s, h, err)
