@@ -539,9 +539,7 @@ def run_kv_variant(args):
     value is the KV-read bandwidth of the keys actually attended; the R = 0
     path on the same inputs runs in alternating blocks beside it."""
     if args.impl == "reference":
-        print(json.dumps({"impl": "reference", "unavailable":
-                          "the reference arm times the contiguous decode only"}))
-        return 0
+        return run_kv_variant_reference(args)
     from parameterized_local_linear_b200 import binding
     dist = Dist(args.gpus)
     dist.init_gpu()
@@ -701,6 +699,39 @@ def run_kv_variant(args):
     if dist.rank == 0:
         print(json.dumps(line))
     dist.close()
+    return 0
+
+
+def run_kv_variant_reference(args):
+    """The reference arm of the paged / block-sparse lines: the fp64 oracle
+    (gathering the same keys) on the first batch rows of the same seeded
+    workload, on the host (rank 0 only)."""
+    if int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    w = inputs.WORKLOADS[args.workload]
+    rows = min(w.B, 16)  # the inputs of the first rows only, drawn on the host
+    wsub = inputs.Workload(w.name, rows, w.Hq, w.Hkv, w.D, w.Lmax, w.dtype, w.seed, w.lengths,
+                           w.r_scale, w.k_offset_std, w.scale)
+    x = (inputs.make_paged(wsub, args.page_size, "cpu") if args.kv_mode == "paged"
+         else inputs.make_block_sparse(wsub, args.density, "cpu"))
+    per_step = min(5.0, 120.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        kv_variant_oracle_sample(args, wsub, x, per_step)
+    vals, t0 = [], time.perf_counter()
+    for _ in range(args.steps):
+        vals.append(kv_variant_oracle_sample(args, wsub, x, per_step))
+    secs = time.perf_counter() - t0
+    value = statistics.mean(v["value"] for v in vals)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": secs / max(1, args.steps) * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": workload_desc(w) + f"; {args.kv_mode}",
+                       "parallelism": "rank 0 only (host CPU)"},
+            "cpu_baseline": dict(vals[-1], value=value),
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
     return 0
 
 
