@@ -57,8 +57,11 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=None)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(inputs.WORKLOADS), default="qwen")
-    ap.add_argument("--num-splits", type=int, default=0)
+    ap.add_argument("--workload", "--config", choices=sorted(inputs.WORKLOADS), default="qwen")
+    ap.add_argument("--num-splits", "--splits", type=int, default=0)
+    ap.add_argument("--out-dtype", choices=["bf16", "f32"], default="bf16",
+                    help="decode output: bf16, or the fp32 debug output")
+    ap.add_argument("--seed", type=int, default=None, help="override the workload's seed")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch size (for profiling a smaller copy)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
@@ -102,7 +105,7 @@ def workload_desc(w: inputs.Workload) -> str:
     lens = {"full": f"L={w.Lmax}", "uniform": f"L~U[1,{w.Lmax}]"}.get(
         w.lengths if isinstance(w.lengths, str) else "", f"L={list(w.lengths)}")
     return (f"{w.name}: Parallax decode B={w.B} Hq={w.Hq} Hkv={w.Hkv} D={w.D} {lens} "
-            f"Lmax={w.Lmax} {str(w.dtype).replace('torch.', '')}")
+            f"Lmax={w.Lmax} {str(w.dtype).replace('torch.', '')} seed={w.seed}")
 
 
 def measured_peaks():
@@ -796,9 +799,11 @@ def main():
     dev = torch.device("cuda", torch.cuda.current_device())
     binding.load_library()
     w = inputs.WORKLOADS[args.workload]
-    if args.batch is not None:
-        w = inputs.Workload(w.name + f"-B{args.batch}", args.batch, w.Hq, w.Hkv, w.D, w.Lmax,
-                            w.dtype, w.seed, w.lengths, w.r_scale, w.k_offset_std, w.scale)
+    if args.batch is not None or args.seed is not None:
+        w = inputs.Workload(w.name + (f"-B{args.batch}" if args.batch is not None else ""),
+                            args.batch if args.batch is not None else w.B, w.Hq, w.Hkv, w.D,
+                            w.Lmax, w.dtype, args.seed if args.seed is not None else w.seed,
+                            w.lengths, w.r_scale, w.k_offset_std, w.scale)
     stream = torch.cuda.Stream(device=dev)  # graphs can not be captured on the legacy stream
     torch.cuda.set_stream(stream)
 
@@ -813,7 +818,8 @@ def main():
         l2_note = f"inputs ({w.kv_bytes_full() / 1e9:.1f} GB of K/V) larger than L2"
     bufs = [x] + [{k: (v.clone() if torch.is_tensor(v) else v) for k, v in x.items()}
                   for _ in range(nbuf - 1)]
-    out = torch.empty((w.B, w.Hq, w.D), device=dev, dtype=torch.bfloat16)
+    out_dtype = torch.float32 if args.out_dtype == "f32" else torch.bfloat16
+    out = torch.empty((w.B, w.Hq, w.D), device=dev, dtype=out_dtype)
     P = args.num_splits if args.num_splits > 0 else binding.parallax_choose_splits(w.B, w.Hkv, w.Lmax)
     ws = binding.Workspace(w.B, w.Hq, w.Hkv, w.D, w.Lmax, P, device=dev)
 
@@ -973,8 +979,23 @@ def main():
     h2d = host_block.numel()
     d2h = out_host.numel() * out_host.element_size()
 
-    # ---- CPU oracle baseline (rank 0, N = 1 only) ----
-    cpu = None
+    # ---- latency distribution, the pages' method: q50 (q05, q95) over trials ----
+    q_stats = None
+    if use_graphs:
+        per_trial = []
+        for _ in range(20):
+            a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            run_plx(nbuf * max(1, 50 // nbuf))
+            b_.record(stream)
+            b_.synchronize()
+            per_trial.append(a.elapsed_time(b_) * 1e3 / (nbuf * max(1, 50 // nbuf)))
+        per_trial.sort()
+        q_stats = {"q05": per_trial[1], "q50": statistics.median(per_trial), "q95": per_trial[-2],
+                   "unit": "us", "method": f"20 trials of {nbuf * max(1, 50 // nbuf)} graph-replayed steps"}
+
+    # ---- CPU oracle baseline and accuracy (rank 0, N = 1 only) ----
+    cpu, accuracy = None, None
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         xh = {k: (v[: min(w.B, 64)].cpu() if torch.is_tensor(v) else v) for k, v in x.items()}
         wsub = inputs.Workload(w.name, min(w.B, 64), w.Hq, w.Hkv, w.D, w.Lmax, w.dtype, w.seed,
@@ -982,6 +1003,18 @@ def main():
         xh["seqlens"] = x["seqlens"][: wsub.B].cpu()
         v, cores, desc, _ = oracle_sample(wsub, xh, args.cpu_seconds)
         cpu = {"value": v, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": desc}
+        # the step's output on the first rows against the oracle (the pages'
+        # bench reports accuracy beside latency)
+        import oracle
+        rows = min(w.B, 8)
+        step(bufs[0])
+        torch.cuda.synchronize()
+        ref = oracle.parallax_decode(xh["q"][:rows], xh["r"][:rows], xh["k"][:rows],
+                                     xh["v"][:rows], xh["seqlens"][:rows], xh["scale"])
+        got = out[:rows].double().cpu().numpy()
+        err = float((abs(got - ref) / abs(ref).clip(min=1.0)).max())
+        accuracy = {"max_scaled_err_vs_oracle": err, "rows": rows,
+                    "out_dtype": args.out_dtype, "tolerance": 1e-4 if args.out_dtype == "f32" else 2e-2}
 
     hbm_peak, peak_src = measured_peaks()
     N = dist.world
@@ -996,7 +1029,8 @@ def main():
         "data": "synthetic",
         "config": {"workload": workload_desc(w), "global_batch": w.B * N, "seq_len": w.Lmax,
                    "parallelism": f"replicas x{N}" if N > 1 else "single GPU",
-                   "num_splits": P, "l2": l2_note, "cuda_graphs": use_graphs},
+                   "num_splits": P, "l2": l2_note, "cuda_graphs": use_graphs,
+                   "out_dtype": args.out_dtype},
         "us_per_step": t_plx / args.steps * 1e6,
         "kv_gbs_frac_of_hbm_peak": gbs / N / hbm_peak,
         "softmax_r0": {"us_per_step": t_soft * 1e6, "kv_gbs": N * step_kv / t_soft / 1e9,
@@ -1014,6 +1048,8 @@ def main():
                      "kernel_us": main_s * 1e6, "launches_timed": main_launches,
                      "algorithmic_bytes_per_launch": main_bytes},
         "cpu_baseline": cpu,
+        "latency_distribution": q_stats,
+        "accuracy": accuracy,
     }
     if dist.rank == 0:
         print(json.dumps(line))

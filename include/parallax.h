@@ -100,7 +100,10 @@ extern "C" {
  * library uses by default: the flattened (batch, kv head, key) range is cut
  * into this many equal parts, so a number of whole waves of the device's SMs
  * is kept busy whatever the batch size and lengths. sm_count <= 0 queries the
- * current device. Returns >= 1, or a negative status for bad arguments.
+ * current device. Returns >= 1, or a negative status for bad arguments. The
+ * environment variable PARALLAX_SPLITS (a positive integer, read once per
+ * process) replaces the heuristic, here and wherever num_splits is 0, for
+ * experiments.
  */
 int parallax_choose_splits(int B, int Hkv, int Lmax, int sm_count);
 

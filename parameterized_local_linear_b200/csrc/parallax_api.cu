@@ -8,6 +8,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstdint>
+#include <cstdlib>
 #include <mutex>
 
 #include "parallax.h"
@@ -68,7 +69,19 @@ int current_sm_count(int* out) {
   return PARALLAX_OK;
 }
 
+// PARALLAX_SPLITS (a positive integer, read once per process) overrides the
+// split heuristic, for experiments; 0 when unset or invalid.
+int env_splits() {
+  static const int value = [] {
+    const char* e = std::getenv("PARALLAX_SPLITS");
+    const long v = e ? std::strtol(e, nullptr, 10) : 0;
+    return (v > 0 && v <= PARALLAX_MAX_SPLITS) ? (int)v : 0;
+  }();
+  return value;
+}
+
 int choose_splits_impl(int B, int Hkv, int Lmax, int sm_count) {
+  if (env_splits() > 0) return env_splits();
   const long long max_keys = (long long)B * Hkv * Lmax;
   const long long slots = (long long)kCtasPerSm * sm_count;
   const long long by_work = std::max(1LL, (max_keys + kMinKeysPerSplit - 1) / kMinKeysPerSplit);

@@ -151,3 +151,19 @@ def test_prefill_argument_errors_before_launch(lib):
     assert call(outd=2) == EDTYPE
     assert call(out=8) == EALIGN
     assert call(wsb=100) == EWS
+
+
+def test_split_env_override():
+    """PARALLAX_SPLITS replaces the split heuristic (read once per process)."""
+    import os
+    import subprocess
+    import sys
+    code = ("import ctypes, sys; lib = ctypes.CDLL(sys.argv[1]); "
+            "print(lib.parallax_choose_splits(1, 8, 4096, 148))")
+    path = binding.library_path()
+    run = lambda env: subprocess.run([sys.executable, "-c", code, path], capture_output=True,
+                                     text=True, env=env, check=True).stdout.strip()
+    base = {k: v for k, v in os.environ.items() if k != "PARALLAX_SPLITS"}
+    assert run(base) == "148"
+    assert run({**base, "PARALLAX_SPLITS": "37"}) == "37"
+    assert run({**base, "PARALLAX_SPLITS": "junk"}) == "148"
