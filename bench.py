@@ -412,6 +412,7 @@ def run_prefill(args):
         cu = torch.tensor([0] + list(torch.tensor(lens).cumsum(0).tolist()), dtype=torch.int32,
                           device=dev)
     out = torch.empty_like(q)
+    out_f32 = out.dtype == torch.float32
     ws = torch.zeros(256, dtype=torch.uint8, device=dev)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     in_bytes = sum(t.numel() * t.element_size() for t in (q, r, k, v, out))
@@ -499,6 +500,34 @@ def run_prefill(args):
     h2d = sum(t.numel() * t.element_size() for t in (hq, hr, hk, hv))
     d2h = out_host.numel() * out_host.element_size()
 
+    # accuracy of this launch configuration against the fp64 oracle on one
+    # sampled slice: the last (batch row, query head) of the dense problem, or
+    # the last packed sequence
+    accuracy = None
+    if dist.rank == 0:
+        import numpy as np
+        import oracle
+        call(0)
+        torch.cuda.synchronize()
+        if lens is None:
+            hh, gg = Hq - 1, (Hq - 1) // (Hq // Hkv)
+            sl = lambda t, i: t[B - 1:B, i:i + 1].cpu()
+            want = oracle.parallax_prefill(sl(q, hh), sl(r, hh), sl(k, gg), sl(v, gg), D ** -0.5,
+                                           True)
+            got = out[B - 1:B, hh:hh + 1].float().cpu().double().numpy()
+            sample = f"batch row {B - 1}, query head {hh}, all {L} rows"
+        else:
+            a0 = int(cu[-2])
+            seg = lambda t: t[a0:].cpu()
+            want = oracle.parallax_varlen_prefill(seg(q), seg(r), seg(k), seg(v),
+                                                  [0, sum(lens) - a0], D ** -0.5, True)
+            got = out[a0:].float().cpu().double().numpy()
+            sample = f"the last sequence ({sum(lens) - a0} rows), all heads"
+        err = float(np.max(np.abs(got - want) / np.maximum(1.0, np.abs(want))))
+        accuracy = {"max_scaled_err": err, "tolerance": 1e-4 if out_f32 else 2e-2,
+                    "pass": bool(np.isfinite(got).all() and err <= (1e-4 if out_f32 else 2e-2)),
+                    "oracle": "fp64", "sample": sample}
+
     cpu = None
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         tf, cores, desc, _ = prefill_oracle_sample(shape, min(10.0, args.cpu_seconds))
@@ -517,6 +546,7 @@ def run_prefill(args):
                        l2=(f"rotate {nbuf} input copies ({nbuf * in_bytes / 1e6:.0f} MB > 2x L2)"
                            if nbuf > 1 else f"inputs ({in_bytes / 1e6:.0f} MB) larger than L2")),
         "softmax_sdpa": sdpa,
+        "accuracy": accuracy,
         "clocks": {k2: clocks[k2] for k2 in ("sm_mhz", "sm_max_mhz", "reasons", "samples")},
         "e2e": {"value": N * flops * k_e2e / t_e2e / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

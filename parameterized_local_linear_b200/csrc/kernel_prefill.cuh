@@ -13,7 +13,8 @@
 // through UMMA.
 //
 // One CTA per (128-row query tile, query head, batch row); late (heavier,
-// causal) tiles first. 320 threads:
+// causal) tiles first across the whole grid, so that the last wave holds the
+// lightest tiles. 320 threads:
 //   warp 8  TMA producer: the Q and R tiles once, then 64-key K and V tiles
 //           into two 3-stage rings (128-byte swizzle, the UMMA operand layout)
 //   warp 9  owns the 512 TMEM columns and issues every UMMA (one lane), in
@@ -25,7 +26,10 @@
 //           32 keys of e and e*s as bf16 hi + lo pairs into the P operand in
 //           TMEM; e and e*s are first rounded to 17 significant bits, so hi +
 //           lo is exact and l, b (summed from the same values) stay consistent
-//           with the weights the products apply. O is rescaled in TMEM only
+//           with the weights the products apply. (One bf16 per weight is not
+//           enough: the value of key i is weighted by e_i (1 + s_i - b/l), so
+//           a weight's rounding error is multiplied by |s|, which for these
+//           probes reaches tens.) O is rescaled in TMEM only
 //           when the max grows by more than 2^8 (otherwise the stale max keeps
 //           every e <= 2^8); each thread of a row rescales one of O_A, O_C.
 // TMEM columns: S [0,64) T [64,128) P [128,256) (per key half, 64 columns:
@@ -117,7 +121,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   float* const red = reinterpret_cast<float*>(gbase + Geo::kOffRed);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int h = blockIdx.y, b = blockIdx.z, g = h / p.G;
+  // CTA -> (query tile slot, head h, batch row b): one linear index with the
+  // slot slowest (slot 0 is every sequence's last, heaviest causal tile), then
+  // h, then b. Slots run to the longest sequence's tile count.
+  const int hb = p.Hq * p.B, slot = (int)blockIdx.x / hb;
+  const int h = ((int)blockIdx.x - slot * hb) % p.Hq, b = ((int)blockIdx.x - slot * hb) / p.Hq;
+  const int g = h / p.G;
   // this sequence: its length L and, packed, its first row s0
   int L = p.L, s0 = 0;
   if (VARLEN) {
@@ -125,12 +134,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     s0 = min(max(a, 0), p.total);
     L = min(max(e, s0), p.total) - s0;
     const bool bad = s0 != a || s0 + L != e;  // outside [0, total] or decreasing
-    if (tid == 0 && blockIdx.x == 0 && h == 0 && (bad || (L + kPfRows - 1) / kPfRows > (int)gridDim.x))
+    if (tid == 0 && slot == 0 && h == 0 && (bad || (L + kPfRows - 1) / kPfRows > p.num_qt))
       atomicOr(p.status, 2u /* PARALLAX_DEVICE_STATUS_SEQLEN_CLAMPED */);
   }
   const int num_qt = VARLEN ? (L + kPfRows - 1) / kPfRows : p.num_qt;
-  if ((int)blockIdx.x >= num_qt) return;  // shorter sequence: nothing for this CTA
-  const int qt = num_qt - 1 - (int)blockIdx.x;  // heavy causal tiles first
+  if (slot >= num_qt) return;  // shorter sequence: nothing for this CTA
+  const int qt = num_qt - 1 - slot;  // heavy causal tiles first
   const int q0 = qt * kPfRows;
   const int kend = p.causal ? min(L, q0 + kPfRows) : L;  // keys this tile can see
   const int nkt = (kend + kPfKeys - 1) / kPfKeys;

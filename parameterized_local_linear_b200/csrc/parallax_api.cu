@@ -569,7 +569,10 @@ int launch_prefill(const void* q, const void* r, const void* k, const void* v,
     if (st != PARALLAX_OK) return st;
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)grid_x, (unsigned)prm.Hq, (unsigned)prm.B);
+  // one linear index over tile slots x Hq x B (slot slowest)
+  const long long lin = (long long)grid_x * prm.Hq * prm.B;
+  if (lin > 0x7fffffffLL) return PARALLAX_ERR_BAD_SHAPE;
+  cfg.gridDim = dim3((unsigned)lin);
   cfg.blockDim = dim3(kPfThreads);
   cfg.dynamicSmemBytes = PfGeom<D>::kSmem;
   cfg.stream = stream;
@@ -673,12 +676,12 @@ extern "C" int parallax_varlen_prefill(const void* q, const void* r, const void*
   prm.Hkv = Hkv;
   prm.G = Hq / Hkv;
   prm.L = 0;
+  prm.num_qt = (max_seqlen + kPfRows - 1) / kPfRows;  // tile slots: the longest sequence's
   prm.total = total_tokens;
   prm.causal = causal != 0;
   prm.scale_log2 = (float)((double)scale * 1.4426950408889634);
   prm.timeout_ns = kDefaultTimeoutNs;
-  return dispatch_prefill<true>(q, r, k, v, prm, D, out_dtype == PARALLAX_DTYPE_F32,
-                                (max_seqlen + kPfRows - 1) / kPfRows,
+  return dispatch_prefill<true>(q, r, k, v, prm, D, out_dtype == PARALLAX_DTYPE_F32, prm.num_qt,
                                 static_cast<cudaStream_t>(stream));
 }
 

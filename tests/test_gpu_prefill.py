@@ -65,11 +65,14 @@ def test_prefill_full_size_sampled():
     finite."""
     B, Hq, Hkv, L, D = 4, 16, 8, 4096, 128
     q, r, k, v = make(B, Hq, Hkv, L, D, seed=7)
-    got = binding.parallax_prefill(q, r, k, v, out_dtype=torch.float32)
-    assert bool(torch.isfinite(got).all())
+    outs = {dt: binding.parallax_prefill(q, r, k, v, out_dtype=dt)
+            for dt in (torch.bfloat16, torch.float32)}  # bf16: the bench's configuration
+    for dt, got in outs.items():
+        assert bool(torch.isfinite(got).all()), dt
     for b, h in ((0, 0), (3, 15)):
         g = h // (Hq // Hkv)
         sl = lambda t, i: t[b:b + 1, i:i + 1]
         want = oracle.parallax_prefill(sl(q, h), sl(r, h), sl(k, g), sl(v, g), D ** -0.5, True)
-        err = scaled_error(got[b:b + 1, h:h + 1], want)
-        assert err <= TOL[torch.float32], (b, h, err)
+        for dt, got in outs.items():
+            err = scaled_error(got[b:b + 1, h:h + 1], want)
+            assert err <= TOL[dt], (b, h, dt, err)
