@@ -210,3 +210,28 @@ def test_full_size_sampled(name):
     finally:
         del x
         torch.cuda.empty_cache()
+
+
+def test_merge_many_pieces_and_workspace_reuse():
+    """Sequences cut into 2 to ~250 pieces (more than one register chunk of
+    partial records in the merge), a keyless sequence among them, the probe
+    and the softmax kernel, and one workspace reused across calls and split
+    counts: every call writes the records it reads."""
+    w = inputs.custom_workload("merge", B=4, Hq=8, Hkv=2, D=128, Lmax=3000, lengths="uniform",
+                               seed=41)
+    x = inputs.make_inputs(w, device="cuda")
+    x["seqlens"][2] = 0  # no keys: o = 0, written by the partition that covers row 2
+    ref = ref_parallax(x)
+    soft = ref_softmax(x)
+    ws = binding.Workspace(4, 8, 2, 128, 3000, num_splits=1000)
+    for splits in (3, 17, 160, 1000):
+        outs = [run(x, torch.float32, num_splits=splits, ws=ws) for _ in range(3)]
+        for o in outs[1:]:
+            assert torch.equal(o, outs[0]), f"{splits} splits: calls differ"
+        assert_close(outs[0], ref, 1e-4, f"{splits} splits")
+        assert float(outs[0][2].abs().max()) == 0.0
+        b = binding.parallax_softmax_decode(x["q"], x["k"], x["v"], x["seqlens"],
+                                            scale=x["scale"], out_dtype=torch.float32,
+                                            num_splits=splits, workspace=ws)
+        assert_close(b, soft, 1e-4, f"softmax, {splits} splits")
+    assert ws.status() == (0, 0)
