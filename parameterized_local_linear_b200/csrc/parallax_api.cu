@@ -248,7 +248,7 @@ int launch_tc(const Call& c, const DecodeParams& prm, int P) {
                                                                         : PARALLAX_ERR_CUDA;
 }
 
-template <typename T, bool PROBE, bool OUT_F32>
+template <typename T, int D, bool PROBE, bool OUT_F32>
 int launch_generic(const Call& c, const DecodeParams& prm, int P) {
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -259,7 +259,7 @@ int launch_generic(const Call& c, const DecodeParams& prm, int P) {
   cfg.stream = c.stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, parallax_generic_kernel<T, PROBE, OUT_F32>, prm) == cudaSuccess
+  return cudaLaunchKernelEx(&cfg, parallax_generic_kernel<T, D, PROBE, OUT_F32>, prm) == cudaSuccess
              ? PARALLAX_OK
              : PARALLAX_ERR_CUDA;
 }
@@ -287,8 +287,11 @@ int launch_split_kv(const Call& c, const DecodeParams& prm, int P) {
     if (c.D == 128) return launch_tc<128, PROBE, OUT_F32>(c, prm, P);
     return launch_tc<64, PROBE, OUT_F32>(c, prm, P);
   }
-  if (c.in_dtype == PARALLAX_DTYPE_BF16) return launch_generic<__nv_bfloat16, PROBE, OUT_F32>(c, prm, P);
-  return launch_generic<float, PROBE, OUT_F32>(c, prm, P);
+  if (c.in_dtype == PARALLAX_DTYPE_BF16)
+    return c.D == 128 ? launch_generic<__nv_bfloat16, 128, PROBE, OUT_F32>(c, prm, P)
+                      : launch_generic<__nv_bfloat16, 64, PROBE, OUT_F32>(c, prm, P);
+  return c.D == 128 ? launch_generic<float, 128, PROBE, OUT_F32>(c, prm, P)
+                    : launch_generic<float, 64, PROBE, OUT_F32>(c, prm, P);
 }
 
 template <bool PROBE, bool OUT_F32>
