@@ -997,12 +997,31 @@ def main():
     out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     k_e2e = min(args.steps, 2000 if use_graphs else args.steps)
 
-    def run_e2e(k):
-        for i in range(k):
-            blk, b = dev_sets[i % nbuf]
-            blk.copy_(host_block, non_blocking=True)
-            step(b)
-            out_host.copy_(out, non_blocking=True)
+    def e2e_step(i):
+        blk, b = dev_sets[i % nbuf]
+        blk.copy_(host_block, non_blocking=True)
+        step(b)
+        out_host.copy_(out, non_blocking=True)
+
+    if use_graphs:
+        # the same copies and launches, replayed from a CUDA graph as the
+        # device-resident steps are (a decode loop captures its copies too)
+        for i in range(nbuf):
+            e2e_step(i)
+        torch.cuda.synchronize()
+        g_e2e = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_e2e, stream=stream):
+            for i in range(nbuf):
+                e2e_step(i)
+        k_e2e = max(nbuf, k_e2e // nbuf * nbuf)
+
+        def run_e2e(k):
+            for _ in range(k // nbuf):
+                g_e2e.replay()
+    else:
+        def run_e2e(k):
+            for i in range(k):
+                e2e_step(i)
 
     t_e2e = timed(run_e2e, k_e2e, min(args.warmup, 50))
     step(bufs[0])  # leave the resident buffers' result behind

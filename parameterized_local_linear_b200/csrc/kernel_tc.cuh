@@ -1,17 +1,17 @@
 // Split-KV Parallax decode kernel for bf16 caches (sm_100a).
 //
 // One CTA per partition of the flattened key range (see partition.cuh),
-// persistent over the pieces of that range. Warp 4 is the producer: one lane
+// persistent over the pieces of that range. Warp 8 is the producer: one lane
 // streams 64-key K and V tiles of the current item with one TMA each (5-D
 // tensor maps {64 dims, keys, D/64 halves, kv heads, batch rows} over either
 // cache layout, 128-byte swizzle, no multicast) into a ring of shared-memory
-// stages guarded by full/empty mbarriers. Warp 8 is the producer; warps 0..7
-// consume in two groups of four that take alternate stages (two tiles in
-// flight through the math at once): warp w owns keys 16 (w % 4) .. +15 of its
-// group's stages and keeps its own online accumulators, so the consumer warps
-// never synchronise inside the key loop. They read the q (and r) rows of the item's
-// GQA group straight into mma fragments from global memory, overlapped with
-// the first K/V tile's flight.
+// stages guarded by full/empty mbarriers. Warps 0..7 consume in two groups of
+// four that take alternate stages (two tiles in flight through the math at
+// once): warp w owns keys 16 (w % 4) .. +15 of its group's stages and keeps its
+// own online accumulators, so the consumer warps never synchronise inside the
+// key loop. They read the q (and r) rows of the item's GQA group straight into
+// mma fragments from global memory, overlapped with the first K/V tile's
+// flight.
 //
 // The method streams the same K/V tiles as FlashAttention and does twice its
 // work per byte ("Parallax: Parameterized Local Linear Attention for Language

@@ -26,7 +26,7 @@ namespace {
 
 constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;  // 2 s per wait
 constexpr long long kMinKeysPerSplit = 128;  // smallest key range worth a CTA (two tiles)
-constexpr int kCtasPerSm = 1;                // split-KV CTAs per SM (96 KB ring each)
+constexpr int kCtasPerSm = 1;                // split-KV CTAs per SM (a 96-128 KB ring each)
 
 struct Call {
   int phases;  // bit 0: split-KV kernel, bit 1: merge kernel
