@@ -196,7 +196,8 @@ int parallax_decode_phase(int phase, int probe, const void* q, const void* r,
  *  - A page id outside [0, num_pages) is not read: its keys are left out and
  *    PARALLAX_DEVICE_STATUS_SEQLEN_CLAMPED is set.
  *  - probe != 0: the Parallax output (r required); probe == 0: R = 0 softmax.
- *  - bf16 inputs only; query heads per kv head at most 4 (probe) or 8.
+ *  - bf16 inputs; any query-head group (groups of more than 4 query heads per
+ *    kv head with the probe, or 8 without, go through the generic kernel).
  *  - Workspace: parallax_decode_workspace_bytes(B, Hq, Hkv, D,
  *    max_pages_per_seq * page_size, num_splits). Other rules as parallax_decode.
  */
@@ -218,7 +219,7 @@ int parallax_decode_paged(const void* q, const void* r, const void* k_pages, con
  *  - A block id outside [0, ceil(Lmax / 64)) or a count outside [0,
  *    max_blocks] is clamped away and sets PARALLAX_DEVICE_STATUS_SEQLEN_CLAMPED.
  *  - A block listed twice is attended twice (its keys count twice).
- *  - bf16 inputs only; query heads per kv head at most 4 (probe) or 8.
+ *  - bf16 inputs; any query-head group, as parallax_decode_paged.
  *  - Workspace: parallax_decode_workspace_bytes(B, Hq, Hkv, D, 64 * max_blocks,
  *    num_splits). Other rules as parallax_decode.
  */

@@ -5,7 +5,10 @@
 //
 // A piece's keys go through shared memory in chunks of 32, the loads of chunk
 // c + 1 in flight (in registers) while chunk c is processed, for up to four
-// query heads of the group per pass. Warp w scores head w, one key per lane
+// query heads of the group per pass. Paged and block-sparse rows resolve each
+// chunk through tile_source (a chunk never straddles a 64-key tile, since
+// pieces start on whole tiles), and only the attended prefix of a tile is
+// loaded. Warp w scores head w, one key per lane
 // (t = scale*log2(e) q.k, s = r.k; K padded by one float per row so the lanes
 // hit distinct banks), takes the chunk max with shuffles and writes the
 // weights e = 2^(t-m') and e*s; then thread d (< D) updates the accumulators
@@ -68,9 +71,6 @@ __global__ void __launch_bounds__(kGenericThreads)
   cur.init(part, key_space(p), p.B, p.Hkv);
   Piece pc;
   while (cur.next(pc)) {
-    const long long kv0 = pc.b * p.kv_sb + pc.g * p.kv_sh + pc.kbase * p.kv_sk;
-    const T* kb = k + kv0;  // key j of the piece's item: kb + j * kv_sk
-    const T* vb = v + kv0;
     const int nchunks = (pc.len + kGenericChunk - 1) / kGenericChunk;
     for (int h0 = 0; h0 < G; h0 += HP) {
       const int nh = min(HP, G - h0);
@@ -86,19 +86,34 @@ __global__ void __launch_bounds__(kGenericThreads)
       for (int hh = 0; hh < HP; ++hh) l[hh] = bs[hh] = A[hh] = C[hh] = 0.f;
 
       float kr[kPer], vr[kPer];
-      auto load_chunk = [&](int c) {  // chunk c's K and V values of this thread, coalesced
-        const int k0 = pc.i + c * kGenericChunk, nk = min(kGenericChunk, pc.i + pc.len - k0);
+      int nv_next = 0;
+      // chunk c's K and V values of this thread (coalesced), and its count of
+      // attended keys (a prefix of the chunk)
+      auto load_chunk = [&](int c) {
+        const int k0 = pc.i + c * kGenericChunk;  // position in the item's key space
+        int nv = min(kGenericChunk, pc.i + pc.len - k0);
+        long long first;  // element offset of the chunk's first key in K and V
+        if (p.kv_mode == kKvContiguous) {
+          first = pc.b * p.kv_sb + pc.g * p.kv_sh + (long long)(pc.kbase + k0) * p.kv_sk;
+        } else {
+          const int o = k0 & (kRangeAlign - 1);
+          int key, item, nvt;
+          tile_source(p, pc.b, k0 - o, &key, &item, &nvt);
+          nv = max(0, min(nv, nvt - o));
+          first = item * p.kv_sb + pc.g * p.kv_sh + (long long)(key + o) * p.kv_sk;
+        }
 #pragma unroll
         for (int u = 0; u < kPer; ++u) {
           const int idx = tid + u * kGenericThreads, j = idx / D, d = idx % D;
-          const long long off = (long long)(k0 + (j < nk ? j : 0)) * p.kv_sk + d;
-          kr[u] = j < nk ? to_f32(kb[off]) : 0.f;
-          vr[u] = j < nk ? to_f32(vb[off]) : 0.f;
+          const long long off = first + (long long)(j < nv ? j : 0) * p.kv_sk + d;
+          kr[u] = j < nv ? to_f32(k[off]) : 0.f;
+          vr[u] = j < nv ? to_f32(v[off]) : 0.f;
         }
+        nv_next = nv;
       };
       load_chunk(0);
       for (int c = 0; c < nchunks; ++c) {
-        const int nk = min(kGenericChunk, pc.len - c * kGenericChunk);
+        const int nk = nv_next;  // attended keys of this chunk
 #pragma unroll
         for (int u = 0; u < kPer; ++u) {
           const int idx = tid + u * kGenericThreads;
@@ -129,7 +144,8 @@ __global__ void __launch_bounds__(kGenericThreads)
           s_es[warp][lane] = e * (s0 + s1);
           __syncwarp();
           if (lane == 0) {
-            s_alpha[warp] = exp2f(mo - mn);  // mo = -inf on the first chunk: 0
+            // no key attended yet (mo = -inf): the sums are 0, whatever mn is
+            s_alpha[warp] = mo == kNegInf ? 0.f : exp2f(mo - mn);
             s_m[warp] = mn;
           }
         }
@@ -163,7 +179,7 @@ __global__ void __launch_bounds__(kGenericThreads)
         if (hh < nh && tid < D) {
           const size_t row = row0 + (size_t)hh * D;
           if (pc.complete) {
-            const float inv = 1.f / l[hh];
+            const float inv = l[hh] > 0.f ? 1.f / l[hh] : 0.f;  // no attended key: o = 0
             const float vbar = A[hh] * inv;
             const float o = PROBE ? vbar + C[hh] * inv - (bs[hh] * inv) * vbar : vbar;
             if (OUT_F32)

@@ -44,29 +44,7 @@
 
 namespace plx {
 
-// Paged and block-sparse rows: where logical tile k0 (a multiple of 64) of
-// batch row b lives, as (*key, *item) coordinates of the K/V tensor maps, and
-// how many of its keys are attended (*nv, a prefix of the tile). An id outside
-// the pool or the cache gives an empty tile and sets the clamped status bit.
-__device__ __forceinline__ void tile_source(const DecodeParams& p, int b, int k0, int* key,
-                                            int* item, int* nv) {
-  const int n = p.seqlens ? clamp_len(__ldg(p.seqlens + b), p.Lmax) : p.Lmax;
-  if (p.kv_mode == kKvPaged) {
-    const int page = __ldg(p.table + (size_t)b * p.table_stride + k0 / p.page_size);
-    const bool ok = page >= 0 && page < p.num_pages;
-    *key = ok ? k0 % p.page_size : 0;
-    *item = ok ? page : 0;
-    *nv = ok ? max(0, min(kTileKeys, n - k0)) : 0;
-    if (!ok) atomicOr(p.status, 2u /* PARALLAX_DEVICE_STATUS_SEQLEN_CLAMPED */);
-  } else {  // block-sparse: the listed block of the cache row
-    const int blk = __ldg(p.table + (size_t)b * p.table_stride + k0 / kTileKeys);
-    const bool ok = blk >= 0 && (long long)blk * kTileKeys < p.Lmax;
-    *key = ok ? blk * kTileKeys : 0;
-    *item = b;
-    *nv = ok ? max(0, min(kTileKeys, n - blk * kTileKeys)) : 0;
-    if (!ok) atomicOr(p.status, 2u);
-  }
-}
+static_assert(kTileKeys == kRangeAlign, "partition ranges are whole tiles of this kernel");
 
 template <int D, bool PROBE, bool OUT_F32, bool PSPLIT>
 __global__ void __launch_bounds__(kTcThreads, 1)

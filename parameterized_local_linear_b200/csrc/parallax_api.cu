@@ -137,10 +137,7 @@ int validate(const Call& c) {
       return PARALLAX_ERR_BAD_SHAPE;
     if (c.kv_mode == kKvBlockSparse && (long long)c.table_stride * kTileKeys > 0x7fffffffLL)
       return PARALLAX_ERR_BAD_SHAPE;
-    // these rows are served by the TMA kernel only: bf16 inputs, a group that fits it
-    const int G = c.Hkv > 0 ? c.Hq / c.Hkv : 0;
-    if (c.in_dtype != PARALLAX_DTYPE_BF16) return PARALLAX_ERR_UNSUPPORTED_DTYPE;
-    if (c.probe ? 2 * G > 8 : G > 8) return PARALLAX_ERR_BAD_SHAPE;
+    if (c.in_dtype != PARALLAX_DTYPE_BF16) return PARALLAX_ERR_UNSUPPORTED_DTYPE;  // bf16 pools
   }
   if (c.probe && !c.r) return PARALLAX_ERR_NULL_POINTER;
   if (!shape_ok(c.B, c.Hq, c.Hkv, c.D, c.Lmax)) return PARALLAX_ERR_BAD_SHAPE;
@@ -318,7 +315,11 @@ int run(const Call& c) {
   prm.r = c.probe ? c.r : nullptr;
   prm.k = c.k;
   prm.v = c.v;
-  const KvStrides kst = kv_strides(c.kv_layout, c.Hkv, c.Lmax, c.D);
+  // a paged pool [pages][page_size][Hkv][D] is a (kv_len, H, D) cache of
+  // page_size keys per page (the TMA kernel's tensor map views it the same way)
+  const KvStrides kst = c.kv_mode == kKvPaged
+                            ? kv_strides(PARALLAX_KV_BSHD, c.Hkv, c.page_size, c.D)
+                            : kv_strides(c.kv_layout, c.Hkv, c.Lmax, c.D);
   prm.kv_sb = kst.b;
   prm.kv_sh = kst.h;
   prm.kv_sk = kst.k;

@@ -213,6 +213,34 @@ struct PieceCursor {
   }
 };
 
+// Paged and block-sparse rows: where logical 64-key tile k0 (a multiple of 64)
+// of batch row b lives, as (*key, *item): the first key and the batch row (or
+// page) of the tile in the K/V view the split-KV kernels read (the paged pool
+// is viewed as a cache of page_size keys per "row" in the (kv_len, H, D)
+// layout), and how many of its keys are attended (*nv, a prefix of the tile).
+// An id outside the pool or the cache gives an empty tile and sets the
+// clamped status bit.
+template <typename Params>
+__device__ __forceinline__ void tile_source(const Params& p, int b, int k0, int* key, int* item,
+                                            int* nv) {
+  const int n = p.seqlens ? clamp_len(__ldg(p.seqlens + b), p.Lmax) : p.Lmax;
+  if (p.kv_mode == kKvPaged) {
+    const int page = __ldg(p.table + (size_t)b * p.table_stride + k0 / p.page_size);
+    const bool ok = page >= 0 && page < p.num_pages;
+    *key = ok ? k0 % p.page_size : 0;
+    *item = ok ? page : 0;
+    *nv = ok ? max(0, min(kRangeAlign, n - k0)) : 0;
+    if (!ok) atomicOr(p.status, 2u /* PARALLAX_DEVICE_STATUS_SEQLEN_CLAMPED */);
+  } else {  // block-sparse: the listed block of the cache row
+    const int blk = __ldg(p.table + (size_t)b * p.table_stride + k0 / kRangeAlign);
+    const bool ok = blk >= 0 && (long long)blk * kRangeAlign < p.Lmax;
+    *key = ok ? blk * kRangeAlign : 0;
+    *item = b;
+    *nv = ok ? max(0, min(kRangeAlign, n - blk * kRangeAlign)) : 0;
+    if (!ok) atomicOr(p.status, 2u);
+  }
+}
+
 // Slot of the partial record of a piece of partition c.
 __device__ __forceinline__ int piece_slot(int c, bool first) { return 2 * c + (first ? 0 : 1); }
 

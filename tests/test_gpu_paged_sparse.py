@@ -41,16 +41,17 @@ def paged_case(seed, B, Hq, Hkv, D, page_size, max_pages, lens, spare=5):
     return q, r, kp, vp, table, n
 
 
-@pytest.mark.parametrize("D,Hq,Hkv", [(128, 16, 8), (64, 8, 8), (128, 8, 2)])
+@pytest.mark.parametrize("D,Hq,Hkv", [(128, 16, 8), (64, 8, 8), (128, 8, 2), (128, 16, 2),
+                                      (64, 32, 4)])
 @pytest.mark.parametrize("page_size", [64, 256])
 def test_paged_matches_oracle(D, Hq, Hkv, page_size):
+    """G = Hq / Hkv up to 8: groups of more than 4 query heads with the probe
+    (or 8 without) go through the generic kernel, the rest the TMA kernel."""
     max_pages = 4096 // page_size
     lens = [1, 700, 4096]
     q, r, kp, vp, table, n = paged_case(500 + D + page_size, 3, Hq, Hkv, D, page_size,
                                         max_pages, lens)
     for probe in (True, False):
-        if probe and Hq // Hkv > 4:
-            continue
         want = oracle.parallax_decode_paged(q, r, kp, vp, table, n, D ** -0.5, probe=probe)
         for out_dtype in (torch.bfloat16, torch.float32):
             for splits in (0, 1, 7):
@@ -92,8 +93,9 @@ def sparse_case(seed, B, Hq, Hkv, D, Lmax, lens, layout):
 
 @pytest.mark.parametrize("layout", ["bhsd", "bshd"])
 @pytest.mark.parametrize("D", [64, 128])
-def test_block_sparse_matches_oracle(layout, D):
-    B, Hq, Hkv, Lmax, nblk = 4, 16, 8, 4096, 64
+@pytest.mark.parametrize("Hq,Hkv", [(16, 8), (16, 2)])
+def test_block_sparse_matches_oracle(layout, D, Hq, Hkv):
+    B, Lmax, nblk = 4, 4096, 64
     lens = [4096, 1000, 37, 4096]
     q, r, k, v, n = sparse_case(600 + D, B, Hq, Hkv, D, Lmax, lens, layout)
     rng = np.random.default_rng(601)
@@ -121,8 +123,9 @@ def test_block_sparse_matches_oracle(layout, D):
                 assert status_bits(ws) == 0
 
 
-def test_block_sparse_bad_ids_are_flagged():
-    B, Hq, Hkv, D, Lmax = 2, 16, 8, 128, 1024
+@pytest.mark.parametrize("Hq,Hkv", [(16, 8), (16, 2)])
+def test_block_sparse_bad_ids_are_flagged(Hq, Hkv):
+    B, D, Lmax = 2, 128, 1024
     q, r, k, v, n = sparse_case(610, B, Hq, Hkv, D, Lmax, [1024, 1024], "bhsd")
     ids = torch.tensor([[0, 99, 2], [1, 2, 3]], dtype=torch.int32, device="cuda")
     cnt = torch.tensor([3, 5], dtype=torch.int32, device="cuda")  # 5 > max_blocks: clamped
