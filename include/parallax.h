@@ -332,6 +332,28 @@ int parallax_decode_noalloc(const void* q, const void* r, const void* k_cache,
                             void* stream, int Lmax, int in_dtype, int out_dtype,
                             int num_splits);
 
+/*
+ * Stream-ordered copy of `bytes` bytes from src to dst done by a kernel, not
+ * by a DMA engine: for the small per-step transfers of a decode loop (q, r
+ * and the lengths in, the output back), where the fixed latency of a DMA copy
+ * is several times the kernel's own. The pages have no counterpart; it exists
+ * for callers that keep a step's inputs and outputs in host memory.
+ *  - Each pointer is device memory, managed memory, or page-locked host
+ *    memory mapped into the current device's address space (cudaHostAlloc or
+ *    cudaHostRegister memory on a system with unified addressing); host
+ *    pointers are translated to their device mapping (cudaPointerGetAttributes'
+ *    devicePointer). Pageable host
+ *    memory, or a host block not mapped for this device, gives
+ *    PARALLAX_ERR_BAD_SHAPE before anything is launched.
+ *  - Both pointers 16-byte aligned and bytes a multiple of 16
+ *    (PARALLAX_ERR_MISALIGNED otherwise); bytes = 0 launches nothing. The
+ *    ranges must not overlap.
+ *  - Writes to host memory are fenced at system scope before the kernel
+ *    ends, so a host thread that waits for the stream (or a later event on
+ *    it) reads the copied bytes.
+ */
+int parallax_copy(void* dst, const void* src, size_t bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -202,6 +202,23 @@ def _stream(stream) -> int:
     return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
 
 
+def parallax_copy(dst, src, stream=None):
+    """Stream-ordered copy of src into dst by a kernel (parallax_copy): for
+    small per-step transfers between device tensors and page-locked host
+    tensors (pin_memory()), where a DMA copy's fixed latency dominates. Both
+    contiguous, the same number of bytes (a multiple of 16)."""
+    if not (dst.is_contiguous() and src.is_contiguous()):
+        raise ValueError("parallax_copy: tensors must be contiguous")
+    nbytes = dst.numel() * dst.element_size()
+    if src.numel() * src.element_size() != nbytes:
+        raise ValueError("parallax_copy: dst and src differ in size")
+    fn = load_library().parallax_copy
+    fn.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+    fn.restype = ctypes.c_int
+    _check(fn(dst.data_ptr(), src.data_ptr(), nbytes, _stream(stream)), "parallax_copy")
+    return dst
+
+
 def parallax_decode(q, r, k_cache, v_cache, cache_seqlens=None, scale: Optional[float] = None,
                     out=None, out_dtype=None, num_splits: int = 0,
                     workspace: Optional[Workspace] = None, stream=None,

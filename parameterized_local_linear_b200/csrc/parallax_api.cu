@@ -15,6 +15,7 @@
 #include "parallax_testing.h"
 
 #include "common.cuh"
+#include "kernel_copy.cuh"
 #include "kernel_generic.cuh"
 #include "kernel_merge.cuh"
 #include "kernel_prefill.cuh"
@@ -482,6 +483,53 @@ int parallax_decode_phase(int phase, int probe, const void* q, const void* r, co
   return run(make_call(phase, probe != 0, q, r, k_cache, v_cache, cache_seqlens, out, B, Hq, Hkv,
                        D, scale, stream, Lmax, in_dtype, out_dtype, num_splits, workspace,
                        workspace_bytes));
+}
+
+}  // extern "C"
+
+namespace {
+
+// The address a kernel on the current device uses for p (for page-locked host
+// memory, its mapping into the device's address space), and whether p is host
+// memory; false for pageable or unmapped host memory.
+bool device_address(const void* p, void** dev, bool* is_host) {
+  cudaPointerAttributes attr{};
+  if (cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  *is_host = attr.type == cudaMemoryTypeHost;
+  if (attr.type == cudaMemoryTypeDevice || attr.type == cudaMemoryTypeManaged) {
+    *dev = const_cast<void*>(p);
+    return true;
+  }
+  if (attr.type != cudaMemoryTypeHost) return false;  // pageable host memory
+  if (attr.devicePointer == nullptr) return false;    // not mapped for this device
+  *dev = attr.devicePointer;
+  return true;
+}
+
+}  // namespace
+
+extern "C" {
+
+int parallax_copy(void* dst, const void* src, size_t bytes, void* stream) {
+  if (!dst || !src) return PARALLAX_ERR_NULL_POINTER;
+  if (!aligned16(dst) || !aligned16(src) || bytes % 16 != 0) return PARALLAX_ERR_MISALIGNED;
+  if (bytes == 0) return PARALLAX_OK;
+  void *d_dst = nullptr, *d_src = nullptr;
+  bool dst_host = false, src_host = false;
+  if (!device_address(dst, &d_dst, &dst_host) || !device_address(src, &d_src, &src_host))
+    return PARALLAX_ERR_BAD_SHAPE;
+  const long long n16 = (long long)(bytes / 16);
+  int sm = 0;
+  int st = current_sm_count(&sm);
+  if (st != PARALLAX_OK) return st;
+  const long long want = (n16 + kCopyThreads - 1) / kCopyThreads;
+  const unsigned blocks = (unsigned)std::max(1LL, std::min<long long>(want, 4LL * sm));
+  parallax_copy_kernel<<<blocks, kCopyThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint4*>(d_dst), static_cast<const uint4*>(d_src), n16, dst_host ? 1 : 0);
+  return cudaGetLastError() == cudaSuccess ? PARALLAX_OK : PARALLAX_ERR_CUDA;
 }
 
 int parallax_workspace_status(void* workspace, int clear, uint32_t* device_status) {
