@@ -887,7 +887,8 @@ def main():
                   for _ in range(nbuf - 1)]
     out_dtype = torch.float32 if args.out_dtype == "f32" else torch.bfloat16
     out = torch.empty((w.B, w.Hq, w.D), device=dev, dtype=out_dtype)
-    P = args.num_splits if args.num_splits > 0 else binding.parallax_choose_splits(w.B, w.Hkv, w.Lmax)
+    P = (args.num_splits if args.num_splits > 0 else
+         binding.parallax_default_splits(w.B, w.Hq, w.Hkv, w.Lmax, w.dtype))
     ws = binding.Workspace(w.B, w.Hq, w.Hkv, w.D, w.Lmax, P, device=dev)
 
     def step(b, probe=True):

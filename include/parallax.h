@@ -51,8 +51,9 @@
  *  - stream is a cudaStream_t (NULL = legacy default stream). Calls are
  *    stream-ordered and asynchronous: no host synchronisation, no allocation,
  *    so they can be captured in a CUDA graph.
- *  - num_splits: 0 lets parallax_choose_splits pick the number of key-range
- *    partitions for the device; a positive value forces it (1 .. 65536).
+ *  - num_splits: 0 picks the number of key-range partitions for the device
+ *    and the kernel the call runs on (parallax_choose_splits); a positive
+ *    value forces it (1 .. 65536).
  *    Results do not depend on it beyond fp32 rounding, and are bitwise
  *    reproducible for a fixed value and device.
  *  - Return value: PARALLAX_OK (0) or a negative status. Argument errors are
@@ -97,15 +98,30 @@ extern "C" {
 
 /*
  * Number of key-range partitions (CTAs of the persistent split-KV kernel) the
- * library uses by default: the flattened (batch, kv head, key) range is cut
- * into this many equal parts, so a number of whole waves of the device's SMs
- * is kept busy whatever the batch size and lengths. sm_count <= 0 queries the
+ * library uses by default for the TMA kernel (bf16 caches, up to 4 query
+ * heads per kv head with the probe, 8 without): the flattened (batch, kv
+ * head, key) range is cut into this many equal parts of at least 128 keys,
+ * at most one per SM, so every SM streams the same bytes whatever the batch
+ * size and lengths. Calls on the generic kernel (fp32 inputs, larger groups)
+ * take parts of at least 64 keys by default, still at most one per SM; the
+ * workspace size for num_splits = 0 covers both. sm_count <= 0 queries the
  * current device. Returns >= 1, or a negative status for bad arguments. The
  * environment variable PARALLAX_SPLITS (a positive integer, read once per
  * process) replaces the heuristic, here and wherever num_splits is 0, for
  * experiments.
  */
 int parallax_choose_splits(int B, int Hkv, int Lmax, int sm_count);
+
+/*
+ * The partition count a decode call with num_splits = 0 uses: the
+ * parallax_choose_splits count on the TMA kernel's path, the generic
+ * kernel's finer count otherwise (in_dtype PARALLAX_DTYPE_F32, or more than
+ * 4 query heads per kv head with probe != 0, or more than 8 without).
+ * sm_count <= 0 queries the current device. Returns >= 1, or a negative
+ * status for bad arguments.
+ */
+int parallax_default_splits(int B, int Hq, int Hkv, int Lmax, int in_dtype, int probe,
+                            int sm_count);
 
 /*
  * Bytes of workspace one decode call needs: a 256-byte header (the device

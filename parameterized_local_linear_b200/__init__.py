@@ -8,7 +8,7 @@ calling any entry point without the built library or a CUDA device raises.
 __all__ = ["parallax_decode", "parallax_softmax_decode", "parallax_decode_phase", "parallax_decode_ex",
            "parallax_prefill", "parallax_varlen_prefill", "parallax_decode_paged",
            "parallax_decode_block_sparse", "parallax_copy",
-           "parallax_decode_workspace_bytes", "parallax_choose_splits",
+           "parallax_decode_workspace_bytes", "parallax_choose_splits", "parallax_default_splits",
            "parallax_status_string", "parallax_workspace_status", "Workspace"]
 
 

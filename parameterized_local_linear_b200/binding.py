@@ -114,6 +114,19 @@ def parallax_choose_splits(B: int, Hkv: int, Lmax: int, sm_count: int = 0) -> in
     return n
 
 
+def parallax_default_splits(B: int, Hq: int, Hkv: int, Lmax: int, dtype=torch.bfloat16,
+                            probe: bool = True, sm_count: int = 0) -> int:
+    """The partition count a decode call with num_splits=0 uses for these
+    shapes, input dtype and probe setting."""
+    fn = load_library().parallax_default_splits
+    fn.argtypes = [ctypes.c_int] * 7
+    fn.restype = ctypes.c_int
+    n = fn(B, Hq, Hkv, Lmax, _DTYPE_CODE[dtype], int(bool(probe)), sm_count)
+    if n < 1:
+        raise RuntimeError(f"parallax_default_splits failed: {parallax_status_string(n)}")
+    return n
+
+
 def parallax_decode_workspace_bytes(B: int, Hq: int, Hkv: int, D: int, Lmax: int,
                                     num_splits: int = 0) -> int:
     n = load_library().parallax_decode_workspace_bytes(B, Hq, Hkv, D, Lmax, num_splits)

@@ -26,7 +26,12 @@ using namespace plx;
 namespace {
 
 constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;  // 2 s per wait
-constexpr long long kMinKeysPerSplit = 128;  // smallest key range worth a CTA (two tiles)
+constexpr long long kMinKeysPerSplit = 128;  // smallest key range worth a TMA-kernel CTA (two tiles)
+// The generic kernel walks a CTA's keys in serial chunks of 32, so it takes
+// ranges half as long (the fp32 tiny decode: 17.8 us per step at 128 keys
+// per split, 11.5 us at 64; the TMA kernel is faster at 128: 6.6 vs 6.9 us
+// for 8192 keys).
+constexpr long long kMinKeysPerSplitGeneric = 64;
 constexpr int kCtasPerSm = 1;                // split-KV CTAs per SM (a 96-128 KB ring each)
 
 struct Call {
@@ -81,11 +86,12 @@ int env_splits() {
   return value;
 }
 
-int choose_splits_impl(int B, int Hkv, int Lmax, int sm_count) {
+int choose_splits_impl(int B, int Hkv, int Lmax, int sm_count,
+                       long long keys_per_split = kMinKeysPerSplit) {
   if (env_splits() > 0) return env_splits();
   const long long max_keys = (long long)B * Hkv * Lmax;
   const long long slots = (long long)kCtasPerSm * sm_count;
-  const long long by_work = std::max(1LL, (max_keys + kMinKeysPerSplit - 1) / kMinKeysPerSplit);
+  const long long by_work = std::max(1LL, (max_keys + keys_per_split - 1) / keys_per_split);
   return (int)std::min(slots, by_work);
 }
 
@@ -104,7 +110,10 @@ size_t workspace_bytes_for(int G, int D, int P) {
 
 int effective_len(int Lmax, int window) { return window > 0 && window < Lmax ? window : Lmax; }
 
-int resolve_splits(int num_splits, int B, int Hkv, int Lmax, int* P) {
+// num_splits, or for 0 the default of the kernel the call runs on (generic:
+// the generic kernel's finer split, which is also what the workspace size
+// function plans for, so that one workspace fits either kernel).
+int resolve_splits(int num_splits, int B, int Hkv, int Lmax, bool generic, int* P) {
   if (num_splits < 0 || num_splits > PARALLAX_MAX_SPLITS) return PARALLAX_ERR_BAD_SPLITS;
   if (num_splits > 0) {
     *P = num_splits;
@@ -113,7 +122,7 @@ int resolve_splits(int num_splits, int B, int Hkv, int Lmax, int* P) {
   int sm = 0;
   const int st = current_sm_count(&sm);
   if (st != PARALLAX_OK) return st;
-  *P = choose_splits_impl(B, Hkv, Lmax, sm);
+  *P = choose_splits_impl(B, Hkv, Lmax, sm, generic ? kMinKeysPerSplitGeneric : kMinKeysPerSplit);
   return PARALLAX_OK;
 }
 
@@ -278,10 +287,16 @@ int launch_merge(const Call& c, const DecodeParams& prm, int P) {
              : PARALLAX_ERR_CUDA;
 }
 
+// The TMA kernel takes bf16 caches whose GQA group (q and r rows with the
+// probe) fits its 8 mma columns; everything else runs on the generic kernel.
+bool tma_path(const Call& c) {
+  const int G = c.Hkv > 0 ? c.Hq / c.Hkv : 0;
+  return c.in_dtype == PARALLAX_DTYPE_BF16 && (c.probe ? 2 * G <= 8 : G <= 8);
+}
+
 template <bool PROBE, bool OUT_F32>
 int launch_split_kv(const Call& c, const DecodeParams& prm, int P) {
-  const bool tc_ok = c.in_dtype == PARALLAX_DTYPE_BF16 && (PROBE ? 2 * prm.G <= 8 : prm.G <= 8);
-  if (tc_ok) {
+  if (tma_path(c)) {
     if (c.D == 128) return launch_tc<128, PROBE, OUT_F32>(c, prm, P);
     return launch_tc<64, PROBE, OUT_F32>(c, prm, P);
   }
@@ -306,7 +321,8 @@ int run(const Call& c) {
   int st = validate(c);
   if (st != PARALLAX_OK) return st;
   int P = 0;
-  if ((st = resolve_splits(c.num_splits, c.B, c.Hkv, planned_len(c), &P)) != PARALLAX_OK)
+  if ((st = resolve_splits(c.num_splits, c.B, c.Hkv, planned_len(c), !tma_path(c), &P)) !=
+      PARALLAX_OK)
     return st;
   const int G = c.Hq / c.Hkv;
   if (c.ws_bytes < workspace_bytes_for(G, c.D, P)) return PARALLAX_ERR_WORKSPACE_TOO_SMALL;
@@ -401,10 +417,28 @@ int parallax_choose_splits(int B, int Hkv, int Lmax, int sm_count) {
   return choose_splits_impl(B, Hkv, Lmax, sm_count);
 }
 
+int parallax_default_splits(int B, int Hq, int Hkv, int Lmax, int in_dtype, int probe,
+                            int sm_count) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || Lmax < 1 || Hq % Hkv != 0) return PARALLAX_ERR_BAD_SHAPE;
+  if (in_dtype != PARALLAX_DTYPE_BF16 && in_dtype != PARALLAX_DTYPE_F32)
+    return PARALLAX_ERR_UNSUPPORTED_DTYPE;
+  if (sm_count <= 0) {
+    const int st = current_sm_count(&sm_count);
+    if (st != PARALLAX_OK) return st;
+  }
+  Call c{};
+  c.Hq = Hq;
+  c.Hkv = Hkv;
+  c.in_dtype = in_dtype;
+  c.probe = probe != 0;
+  return choose_splits_impl(B, Hkv, Lmax, sm_count,
+                            tma_path(c) ? kMinKeysPerSplit : kMinKeysPerSplitGeneric);
+}
+
 size_t parallax_decode_workspace_bytes(int B, int Hq, int Hkv, int D, int Lmax, int num_splits) {
   if (!shape_ok(B, Hq, Hkv, D, Lmax) || (D != 64 && D != 128)) return 0;
   int P = 0;
-  if (resolve_splits(num_splits, B, Hkv, Lmax, &P) != PARALLAX_OK) return 0;
+  if (resolve_splits(num_splits, B, Hkv, Lmax, true, &P) != PARALLAX_OK) return 0;
   return workspace_bytes_for(Hq / Hkv, D, P);
 }
 
@@ -797,7 +831,7 @@ extern "C" int parallax_decode_noalloc(const void* q, const void* r, const void*
                      stream, Lmax, in_dtype, out_dtype, num_splits, scratch, kNoallocScratchBytes);
   if ((st = validate(c)) != PARALLAX_OK) return st;
   int P = 0;
-  if ((st = resolve_splits(num_splits, B, Hkv, Lmax, &P)) != PARALLAX_OK) return st;
+  if ((st = resolve_splits(num_splits, B, Hkv, Lmax, !tma_path(c), &P)) != PARALLAX_OK) return st;
   if (workspace_bytes_for(Hq / Hkv, D, P) > kNoallocScratchBytes) return PARALLAX_ERR_SCRATCH_LIMIT;
   // The array keeps the previous call's contents: the status word must start
   // at zero; the partial records are always written before they are read.

@@ -66,6 +66,16 @@ def test_choose_splits_host_only(lib):
     assert lib.parallax_choose_splits(1, 1, 1, 148) == 1
     assert lib.parallax_choose_splits(2, 2, 128, 148) == 4  # 512 keys / 128
     assert lib.parallax_choose_splits(0, 8, 4096, 148) == ESHAPE
+    # the default a call with num_splits = 0 uses: the generic kernel's finer count
+    # for fp32 inputs or large groups (keys / 64), else the count above
+    f = lib.parallax_default_splits
+    bf16, f32 = 0, 1
+    assert f(2, 4, 2, 128, bf16, 1, 148) == 4     # TMA kernel: 512 keys / 128
+    assert f(2, 4, 2, 128, f32, 1, 148) == 8      # generic (fp32): 512 keys / 64
+    assert f(1, 16, 2, 1024, bf16, 1, 148) == 32  # G = 8 with the probe: generic
+    assert f(1, 16, 2, 1024, bf16, 0, 148) == 16  # G = 8 without: TMA kernel
+    assert f(1, 16, 8, 4096, f32, 1, 148) == 148  # capped at one CTA per SM
+    assert f(1, 12, 8, 4096, bf16, 1, 148) == ESHAPE
 
 
 def test_workspace_bytes_host_only(lib):
