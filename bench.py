@@ -1030,8 +1030,8 @@ def main():
     host_block = host_block.pin_memory()
     dev_sets = []
     for b in bufs:
-        blk, (dq, dr, dsl) = packed_views([x["q"], x["r"], x["seqlens"]], dev)
-        dev_sets.append((blk, {**b, "q": dq, "r": dr, "seqlens": dsl}))
+        dev_blk, (dq, dr, dsl) = packed_views([x["q"], x["r"], x["seqlens"]], dev)
+        dev_sets.append((dev_blk, {**b, "q": dq, "r": dr, "seqlens": dsl}))
     out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     k_e2e = min(args.steps, 2000 if use_graphs else args.steps)
 
@@ -1043,11 +1043,11 @@ def main():
                 else "cudaMemcpyAsync (DMA)")
 
     def e2e_step(i):
-        blk, b = dev_sets[i % nbuf]
+        dev_blk, b = dev_sets[i % nbuf]
         if small:
-            binding.parallax_copy(blk, host_block, stream=stream)
+            binding.parallax_copy(dev_blk, host_block, stream=stream)
         else:
-            blk.copy_(host_block, non_blocking=True)
+            dev_blk.copy_(host_block, non_blocking=True)
         step(b)
         if small:
             binding.parallax_copy(out_host, out, stream=stream)
