@@ -57,7 +57,7 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=None)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", "--config", choices=sorted(inputs.WORKLOADS), default="qwen")
+    ap.add_argument("--workload", "--config", choices=sorted(inputs.WORKLOADS), default="large")
     ap.add_argument("--num-splits", "--splits", type=int, default=0)
     ap.add_argument("--out-dtype", choices=["bf16", "f32"], default="bf16",
                     help="decode output: bf16, or the fp32 debug output")
@@ -67,6 +67,8 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="bound of the CPU oracle baseline sample (seconds)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-companion", action="store_true",
+                    help="skip the Qwen B=1 step measured beside a larger workload")
     ap.add_argument("--kv-mode", choices=["contiguous", "paged", "block_sparse"],
                     default="contiguous", help="where the decode reads its keys from")
     ap.add_argument("--page-size", type=int, default=256)
@@ -129,12 +131,25 @@ def measured_bf16_peak():
         return FALLBACK_BF16_TFLOPS, "fallback"
 
 
-def profiled_traffic():
-    """Per-launch DRAM traffic of the split-KV kernel from the committed ncu
-    summary, if it was taken on the current kernel source."""
-    path = os.path.join(ROOT, "profiles", "parallax_tc_kernel_qwen.md")
+# ncu summaries whose traffic line the bench reports, per workload: (file,
+# batch rows the capture ran). A capture on fewer rows than the workload is
+# scaled by the rows processed (every row of these workloads has the same
+# length, so the split-KV kernel's traffic grows in proportion).
+PROFILE_FOR = {"qwen": ("parallax_tc_kernel_qwen.md", 1),
+               "large": ("parallax_tc_kernel_large_B64.md", 64)}
+
+
+def profiled_traffic(w):
+    """Per-launch DRAM traffic (read + write) of the split-KV kernel from the
+    committed ncu summary of this workload, if it was taken on the current
+    kernel source; scaled to the workload's batch when captured on fewer
+    rows. None otherwise."""
+    name = w.name.split("-")[0]
+    if name not in PROFILE_FOR or w.name != name:
+        return None
+    fname, rows = PROFILE_FOR[name]
     try:
-        text = open(path).read()
+        text = open(os.path.join(ROOT, "profiles", fname)).read()
     except OSError:
         return None
     h = hashlib.sha256()
@@ -145,7 +160,7 @@ def profiled_traffic():
     m_traffic = re.search(r"traffic_bytes_per_launch:\s*([0-9]+)", text)
     if not m_hash or not m_traffic or m_hash.group(1) != src_hash:
         return None
-    return int(m_traffic.group(1))
+    return int(m_traffic.group(1)) * w.B // rows
 
 
 class ClockSampler:
@@ -156,7 +171,7 @@ class ClockSampler:
                0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
                0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
 
-    def __init__(self, device_index: int, period_s: float = 0.02):
+    def __init__(self, device_index: int, period_s: float = 0.005):
         self.samples, self.period, self._stop = [], period_s, threading.Event()
         self.ok = False
         try:
@@ -437,21 +452,7 @@ def run_prefill(args):
                 events[i][1].record(stream)
 
     def timed(fn, k_steps, w_steps, sampler=None):
-        fn(w_steps)
-        torch.cuda.synchronize()
-        dist.barrier()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        if sampler:
-            sampler.__enter__()
-        e0.record(stream)
-        fn(k_steps)
-        e1.record(stream)
-        e1.synchronize()
-        if sampler:
-            sampler.__exit__(None, None, None)
-        torch.cuda.synchronize()
-        dist.barrier()
-        return dist.max(e0.elapsed_time(e1) / 1e3)
+        return timed_steps(dist, stream, fn, k_steps, w_steps, sampler)
 
     sampler = ClockSampler(dev.index)
     t_step = timed(run, args.steps, args.warmup, sampler)
@@ -496,7 +497,7 @@ def run_prefill(args):
             out_host.copy_(out, non_blocking=True)
 
     k_e2e = min(args.steps, 20)
-    t_e2e = timed(run_e2e, k_e2e, 2)
+    t_e2e = timed_plain(dist, stream, run_e2e, k_e2e, 2)
     h2d = sum(t.numel() * t.element_size() for t in (hq, hr, hk, hv))
     d2h = out_host.numel() * out_host.element_size()
 
@@ -644,21 +645,7 @@ def run_kv_variant(args):
             step(probe, i)
 
     def timed(fn, k_steps, w_steps, sampler=None):
-        fn(w_steps)
-        torch.cuda.synchronize()
-        dist.barrier()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        if sampler:
-            sampler.__enter__()
-        e0.record(stream)
-        fn(k_steps)
-        e1.record(stream)
-        e1.synchronize()
-        if sampler:
-            sampler.__exit__(None, None, None)
-        torch.cuda.synchronize()
-        dist.barrier()
-        return dist.max(e0.elapsed_time(e1) / 1e3)
+        return timed_steps(dist, stream, fn, k_steps, w_steps, sampler)
 
     if nbuf > 1:  # whole graph chains only
         args.steps = max(nbuf, args.steps // nbuf * nbuf)
@@ -727,7 +714,7 @@ def run_kv_variant(args):
         def run_e2e(k_steps):
             for i in range(k_steps):
                 e2e_step(i)
-    t_e2e = timed(run_e2e, k_e2e, 2)
+    t_e2e = timed_plain(dist, stream, run_e2e, k_e2e, 2)
     # CPU baseline: the oracle (it gathers the same keys into a dense cache) on
     # the first batch rows, as many as fit in the budget (rank 0, N = 1 only)
     cpu = None
@@ -850,6 +837,204 @@ def kv_variant_oracle_sample(args, w, x, budget_s):
 
 # ------------------------------------------------------------- GPU timing ----
 
+class DecodeRig:
+    """One decode workload resident on the device: its K/V copies (rotated
+    when smaller than twice the L2), output, workspace and split count, and
+    runners for the Parallax and R = 0 steps."""
+
+    def __init__(self, w, dev, stream, out_dtype, num_splits):
+        from parameterized_local_linear_b200 import binding
+        self.binding, self.w, self.dev, self.stream = binding, w, dev, stream
+        self.x = inputs.make_inputs(w, device=dev, pad_value=None)
+        self.step_kv = kv_bytes(self.x)
+        self.l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+        self.nbuf = 1
+        if w.kv_bytes_full() < 2 * self.l2:
+            self.nbuf = max(2, math.ceil(2 * self.l2 / w.kv_bytes_full()))
+            self.l2_note = (f"rotate {self.nbuf} K/V copies "
+                            f"({self.nbuf * w.kv_bytes_full() / 1e6:.0f} MB > 2x L2)")
+        else:
+            self.l2_note = f"inputs ({w.kv_bytes_full() / 1e9:.1f} GB of K/V) larger than L2"
+        x = self.x
+        self.bufs = [x] + [{k: (v.clone() if torch.is_tensor(v) else v) for k, v in x.items()}
+                           for _ in range(self.nbuf - 1)]
+        self.out = torch.empty((w.B, w.Hq, w.D), device=dev, dtype=out_dtype)
+        self.P = (num_splits if num_splits > 0 else
+                  binding.parallax_default_splits(w.B, w.Hq, w.Hkv, w.Lmax, w.dtype))
+        self.ws = binding.Workspace(w.B, w.Hq, w.Hkv, w.D, w.Lmax, self.P, device=dev)
+        self.use_graphs = self.nbuf > 1
+        self.runners = {True: self._make_runner(True), False: self._make_runner(False)}
+
+    def step(self, b, probe=True):
+        bd = self.binding
+        if probe:
+            bd.parallax_decode(b["q"], b["r"], b["k"], b["v"], b["seqlens"], scale=b["scale"],
+                               out=self.out, num_splits=self.P, workspace=self.ws,
+                               stream=self.stream)
+        else:
+            bd.parallax_softmax_decode(b["q"], b["k"], b["v"], b["seqlens"], scale=b["scale"],
+                                       out=self.out, num_splits=self.P, workspace=self.ws,
+                                       stream=self.stream)
+
+    def _make_runner(self, probe):
+        """run(k) enqueues exactly k steps. Graph-replayed workloads replay
+        whole chains of `chain` steps (a multiple of the rotation) and one
+        graph of the remainder; run.prepare(k) captures what run(k) replays,
+        so that no capture falls inside a timed region."""
+        bufs, nbuf = self.bufs, self.nbuf
+        if not self.use_graphs:
+            def run(k):
+                for i in range(k):
+                    self.step(bufs[i % nbuf], probe)
+            run.prepare = lambda k: None
+            return run
+        for b in bufs:  # warm the launch path outside capture
+            self.step(b, probe)
+        torch.cuda.synchronize()
+        graphs = {}
+        chain = nbuf * max(1, 256 // nbuf)
+
+        def graph(n):
+            if n not in graphs:
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=self.stream):
+                    for i in range(n):
+                        self.step(bufs[i % nbuf], probe)
+                graphs[n] = g
+            return graphs[n]
+
+        def prepare(k):
+            if k >= chain:
+                graph(chain)
+            if k % chain:
+                graph(k % chain)
+
+        def run(k):
+            prepare(k)
+            for _ in range(k // chain):
+                graphs[chain].replay()
+            if k % chain:
+                graphs[k % chain].replay()
+        run.prepare = prepare
+        return run
+
+    def host_seconds_per_step(self, probe=True, k=None):
+        """Host time to enqueue one step (the gate in front of a timed region
+        must outlast the enqueueing of the steps behind it)."""
+        run = self.runners[probe]
+        k = k or (256 if self.use_graphs else 4)
+        run.prepare(k)
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        run(k)
+        dt = time.perf_counter() - t0
+        torch.cuda.synchronize()
+        return dt / k
+
+
+def timed_plain(dist, stream, fn, k_steps, w_steps):
+    """W untimed steps, then K steps between two events, enqueued as the host
+    goes (the end-to-end loop: host launch gaps and copies are part of it)."""
+    fn(w_steps)
+    torch.cuda.synchronize()
+    dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    fn(k_steps)
+    e1.record(stream)
+    e1.synchronize()
+    torch.cuda.synchronize()
+    dist.barrier()
+    return dist.max(e0.elapsed_time(e1) / 1e3)
+
+
+def timed_steps(dist, stream, fn, k_steps, w_steps, sampler=None):
+    """W untimed steps, then exactly K steps timed by gated_region (queued
+    behind a sleep kernel), barrier and synchronize on both sides, max over
+    ranks."""
+    fn(w_steps)
+    torch.cuda.synchronize()
+    n = max(1, min(k_steps, 4))
+    t0 = time.perf_counter()
+    fn(n)  # the host's enqueue time per step sizes the gate
+    host = (time.perf_counter() - t0) / n
+    torch.cuda.synchronize()
+    dist.barrier()
+    t = gated_region(stream, lambda: fn(k_steps), host * k_steps, sampler)
+    torch.cuda.synchronize()
+    dist.barrier()
+    return dist.max(t)
+
+
+def gated_region(stream, enqueue, host_s, sampler=None):
+    """Time the launches `enqueue()` issues with CUDA events on `stream`, with
+    the launches queued before the region starts: a sleep kernel holds the
+    stream (torch.cuda._sleep, a fixed cycle count) while the host enqueues,
+    so that host launch gaps do not land in the timed region. Returns
+    seconds between the events."""
+    gate_s = min(0.25, max(0.002, 1.5 * host_s))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda._sleep(int(gate_s * 2.0e9))  # cycles at up to 2 GHz
+    e0.record(stream)
+    enqueue()
+    e1.record(stream)
+    if sampler:
+        sampler.__enter__()
+    e1.synchronize()
+    if sampler:
+        sampler.__exit__(None, None, None)
+    return e0.elapsed_time(e1) / 1e3
+
+
+def same_block_medians(rig, rounds, blk):
+    """The R = 0 comparator: blocks of Parallax and softmax steps alternate,
+    so both see the same power and clock state (B200 runs at its power cap
+    while streaming HBM); each block is a gated region of whole steps."""
+    per = {True: [], False: []}
+    host = {p: rig.host_seconds_per_step(p) for p in (True, False)}
+    for p in (True, False):
+        rig.runners[p].prepare(blk)
+        rig.runners[p](min(blk, 2 * rig.nbuf))
+    torch.cuda.synchronize()
+    for _ in range(rounds):
+        for probe in (True, False):
+            run = rig.runners[probe]
+            per[probe].append(gated_region(rig.stream, lambda: run(blk), host[probe] * blk) / blk)
+    return statistics.median(per[True]), statistics.median(per[False]), per
+
+
+def qwen_companion(dev, stream, dist):
+    """The latency-bound Qwen-3 decode step (B = 1, 16.8 MB of K/V) measured
+    beside the default workload: same-block medians of Parallax and R = 0,
+    and the pages' q05/q50/q95 statistic over trials."""
+    w = inputs.WORKLOADS["qwen"]
+    rig = DecodeRig(w, dev, stream, torch.bfloat16, 0)
+    blk = rig.nbuf * max(1, 800 // rig.nbuf)
+    t_p, t_s, _ = same_block_medians(rig, 8, blk)
+    per_trial = []
+    run = rig.runners[True]
+    n_trial = rig.nbuf * max(1, 50 // rig.nbuf)
+    host = rig.host_seconds_per_step(True)
+    for _ in range(20):
+        per_trial.append(gated_region(stream, lambda: run(n_trial), host * n_trial) / n_trial)
+    per_trial.sort()
+    out = {"workload": workload_desc(w), "num_splits": rig.P, "l2": rig.l2_note,
+           "us_per_step_same_blocks": dist.max(t_p) * 1e6,
+           "softmax_r0_us_per_step": dist.max(t_s) * 1e6,
+           "parallax_over_softmax_latency": t_p / t_s,
+           "kv_gbs_same_blocks": rig.step_kv / dist.max(t_p) / 1e9,
+           "latency_us": {"q05": per_trial[1] * 1e6, "q50": statistics.median(per_trial) * 1e6,
+                          "q95": per_trial[-2] * 1e6},
+           "method": f"8 alternating gated blocks of {blk} graph-replayed steps (medians); "
+                     f"20 trials of {n_trial} steps for the quantiles"}
+    rc, _ = rig.ws.status()
+    if rc != 0:
+        raise SystemExit(f"device status after the qwen step: {rig.binding.parallax_status_string(rc)}")
+    del rig
+    torch.cuda.empty_cache()
+    return out
+
+
 def main():
     args = parse_args()
     if args.prefill:
@@ -874,99 +1059,38 @@ def main():
     stream = torch.cuda.Stream(device=dev)  # graphs can not be captured on the legacy stream
     torch.cuda.set_stream(stream)
 
-    x = inputs.make_inputs(w, device=dev, pad_value=None)
-    step_kv = kv_bytes(x)
-    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    nbuf = 1
-    if w.kv_bytes_full() < 2 * l2:
-        nbuf = max(2, math.ceil(2 * l2 / w.kv_bytes_full()))
-        l2_note = f"rotate {nbuf} K/V copies ({nbuf * w.kv_bytes_full() / 1e6:.0f} MB > 2x L2)"
-    else:
-        l2_note = f"inputs ({w.kv_bytes_full() / 1e9:.1f} GB of K/V) larger than L2"
-    bufs = [x] + [{k: (v.clone() if torch.is_tensor(v) else v) for k, v in x.items()}
-                  for _ in range(nbuf - 1)]
     out_dtype = torch.float32 if args.out_dtype == "f32" else torch.bfloat16
-    out = torch.empty((w.B, w.Hq, w.D), device=dev, dtype=out_dtype)
-    P = (args.num_splits if args.num_splits > 0 else
-         binding.parallax_default_splits(w.B, w.Hq, w.Hkv, w.Lmax, w.dtype))
-    ws = binding.Workspace(w.B, w.Hq, w.Hkv, w.D, w.Lmax, P, device=dev)
+    rig = DecodeRig(w, dev, stream, out_dtype, args.num_splits)
+    x, bufs, nbuf, out, ws, P = rig.x, rig.bufs, rig.nbuf, rig.out, rig.ws, rig.P
+    step, step_kv, use_graphs = rig.step, rig.step_kv, rig.use_graphs
+    run_plx, run_soft = rig.runners[True], rig.runners[False]
 
-    def step(b, probe=True):
-        if probe:
-            binding.parallax_decode(b["q"], b["r"], b["k"], b["v"], b["seqlens"], scale=b["scale"],
-                                    out=out, num_splits=P, workspace=ws, stream=stream)
-        else:
-            binding.parallax_softmax_decode(b["q"], b["k"], b["v"], b["seqlens"],
-                                            scale=b["scale"], out=out, num_splits=P,
-                                            workspace=ws, stream=stream)
-
-    use_graphs = nbuf > 1
-
-    def make_runner(probe):
-        if not use_graphs:
-            def run(k):
-                for i in range(k):
-                    step(bufs[i % nbuf], probe)
-            return run
-        for b in bufs:  # warm the launch path outside capture
-            step(b, probe)
-        torch.cuda.synchronize()
-        chain = torch.cuda.CUDAGraph()
-        singles = []
-        with torch.cuda.graph(chain, stream=stream):
-            for b in bufs:
-                step(b, probe)
-        for b in bufs:
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                step(b, probe)
-            singles.append(g)
-
-        def run(k):
-            for _ in range(k // nbuf):
-                chain.replay()
-            for i in range(k % nbuf):
-                singles[i].replay()
-        return run
-
-    def timed(run, k, w_steps, sampler=None):
-        run(w_steps)
-        torch.cuda.synchronize()
-        dist.barrier()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        if sampler:
-            sampler.__enter__()
-        e0.record(stream)
-        run(k)
-        e1.record(stream)
-        e1.synchronize()
-        if sampler:
-            sampler.__exit__(None, None, None)
-        torch.cuda.synchronize()
-        dist.barrier()
-        return dist.max(e0.elapsed_time(e1) / 1e3)
-
-    run_plx = make_runner(True)
-    run_soft = make_runner(False)
+    # ---- the timed region: exactly K steps after W warm-up steps ----
+    run_plx.prepare(args.steps)
+    run_plx(args.warmup)
+    host_s = rig.host_seconds_per_step(True) * args.steps
+    torch.cuda.synchronize()
+    dist.barrier()
     sampler = ClockSampler(dev.index)
-    t_plx = timed(run_plx, args.steps, args.warmup, sampler)
+    t_plx = dist.max(gated_region(stream, lambda: run_plx(args.steps), host_s, sampler))
+    torch.cuda.synchronize()
+    dist.barrier()
 
-    # The R = 0 comparator: blocks of Parallax and softmax steps alternate, so
-    # both see the same power and clock state (B200 runs at its power cap
-    # while streaming HBM); the ratio is taken from the block medians.
+    # ---- sustained: whole steps over at least one second ----
+    per_step = t_plx / args.steps
+    chain = nbuf * max(1, 256 // nbuf) if use_graphs else 1
+    k_sus = max(args.steps, math.ceil(1.0 / per_step / chain) * chain)
+    run_plx.prepare(k_sus)
+    sus_sampler = ClockSampler(dev.index)
+    torch.cuda.synchronize()
+    dist.barrier()
+    t_sus = dist.max(gated_region(stream, lambda: run_plx(k_sus),
+                                  rig.host_seconds_per_step(True) * k_sus, sus_sampler))
+    sus_clocks = sus_sampler.summary()
+
     blk = nbuf * max(1, 800 // nbuf) if use_graphs else 10
     rounds = 8 if use_graphs else 5
-    run_soft(min(args.warmup, blk))
-    per = {True: [], False: []}
-    for _ in range(rounds):
-        for probe, runner in ((True, run_plx), (False, run_soft)):
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            runner(blk)
-            b.record(stream)
-            b.synchronize()
-            per[probe].append(a.elapsed_time(b) / 1e3 / blk)
-    t_plx_blk, t_soft_blk = statistics.median(per[True]), statistics.median(per[False])
+    t_plx_blk, t_soft_blk, _ = same_block_medians(rig, rounds, blk)
     t_soft = dist.max(t_soft_blk)
     t_plx_blk = dist.max(t_plx_blk)
     rc, bits = ws.status()
@@ -989,14 +1113,12 @@ def main():
         reps = max(1, min(args.steps, 20000) // nbuf)
         for _ in range(3):
             g1.replay()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize()
-        e0.record(stream)
-        for _ in range(reps):
-            g1.replay()
-        e1.record(stream)
-        e1.synchronize()
-        main_s = e0.elapsed_time(e1) / 1e3 / (reps * nbuf)
+
+        def enqueue_p1():
+            for _ in range(reps):
+                g1.replay()
+        main_s = gated_region(stream, enqueue_p1, 1e-5 * reps) / (reps * nbuf)
         main_launches = reps * nbuf
     else:
         nprof = min(args.steps, 50)
@@ -1074,7 +1196,18 @@ def main():
             for i in range(k):
                 e2e_step(i)
 
-    t_e2e = timed(run_e2e, k_e2e, min(args.warmup, 50))
+    # the end-to-end loop is timed as a user runs it: launches and copies
+    # enqueued as the host goes, no gate in front
+    run_e2e(min(args.warmup, 50))
+    torch.cuda.synchronize()
+    dist.barrier()
+    ee0, ee1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ee0.record(stream)
+    run_e2e(k_e2e)
+    ee1.record(stream)
+    ee1.synchronize()
+    dist.barrier()
+    t_e2e = dist.max(ee0.elapsed_time(ee1) / 1e3)
     step(bufs[0])  # leave the resident buffers' result behind
     h2d = host_block.numel()
     d2h = out_host.numel() * out_host.element_size()
@@ -1083,16 +1216,13 @@ def main():
     q_stats = None
     if use_graphs:
         per_trial = []
+        n_trial = nbuf * max(1, 50 // nbuf)
+        host_t = rig.host_seconds_per_step(True) * n_trial
         for _ in range(20):
-            a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            run_plx(nbuf * max(1, 50 // nbuf))
-            b_.record(stream)
-            b_.synchronize()
-            per_trial.append(a.elapsed_time(b_) * 1e3 / (nbuf * max(1, 50 // nbuf)))
+            per_trial.append(gated_region(stream, lambda: run_plx(n_trial), host_t) / n_trial * 1e6)
         per_trial.sort()
         q_stats = {"q05": per_trial[1], "q50": statistics.median(per_trial), "q95": per_trial[-2],
-                   "unit": "us", "method": f"20 trials of {nbuf * max(1, 50 // nbuf)} graph-replayed steps"}
+                   "unit": "us", "method": f"20 trials of {n_trial} graph-replayed steps"}
 
     # ---- CPU oracle baseline and accuracy (rank 0, N = 1 only) ----
     cpu, accuracy = None, None
@@ -1116,6 +1246,12 @@ def main():
         accuracy = {"max_scaled_err_vs_oracle": err, "rows": rows,
                     "out_dtype": args.out_dtype, "tolerance": 1e-4 if args.out_dtype == "f32" else 2e-2}
 
+    # ---- the latency-bound Qwen step beside the default workload ----
+    companion = None
+    if args.workload != "qwen" and not args.no_companion:
+        del dev_sets, host_block, out_host
+        companion = qwen_companion(dev, stream, dist)
+
     hbm_peak, peak_src = measured_peaks()
     N = dist.world
     gbs = replicas.whole_job_rate(args.steps * step_kv, t_plx, N) / 1e9
@@ -1129,27 +1265,36 @@ def main():
         "data": "synthetic",
         "config": {"workload": workload_desc(w), "global_batch": w.B * N, "seq_len": w.Lmax,
                    "parallelism": f"replicas x{N}" if N > 1 else "single GPU",
-                   "num_splits": P, "l2": l2_note, "cuda_graphs": use_graphs,
-                   "out_dtype": args.out_dtype},
+                   "num_splits": P, "l2": rig.l2_note, "cuda_graphs": use_graphs,
+                   "out_dtype": args.out_dtype,
+                   "timing": "CUDA events around exactly K steps, enqueued behind a sleep "
+                             "kernel so that no host launch gap is timed"},
         "us_per_step": t_plx / args.steps * 1e6,
         "kv_gbs_frac_of_hbm_peak": gbs / N / hbm_peak,
+        "sustained": {"steps": k_sus, "seconds": t_sus, "us_per_step": t_sus / k_sus * 1e6,
+                      "value": replicas.whole_job_rate(k_sus * step_kv, t_sus, N) / 1e9,
+                      "unit": "GB/s",
+                      "clocks": {k: sus_clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons",
+                                                            "samples")},
+                      "method": "whole steps over at least one second, one gated region"},
         "softmax_r0": {"us_per_step": t_soft * 1e6, "kv_gbs": N * step_kv / t_soft / 1e9,
                        "parallax_us_per_step_same_blocks": t_plx_blk * 1e6,
                        "parallax_over_softmax_latency": t_plx_blk / t_soft,
-                       "method": f"{rounds} alternating blocks of {blk} steps each, medians"},
+                       "method": f"{rounds} alternating gated blocks of {blk} steps each, medians"},
         "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons", "samples")},
         "e2e": {"value": N * k_e2e * step_kv / t_e2e / 1e9, "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "us_per_step": t_e2e / k_e2e * 1e6, "transfer": transfer},
         "gpu_launches": 2 * args.steps,  # split-KV + merge per step, in the timed region
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": achieved / hbm_peak, "traffic": profiled_traffic(),
+                     "frac": achieved / hbm_peak, "traffic": profiled_traffic(w),
                      "kernel": "parallax_tc_kernel (split-KV)", "peak_source": peak_src,
                      "kernel_us": main_s * 1e6, "launches_timed": main_launches,
                      "algorithmic_bytes_per_launch": main_bytes},
         "cpu_baseline": cpu,
         "latency_distribution": q_stats,
         "accuracy": accuracy,
+        "qwen_step": companion,
     }
     if dist.rank == 0:
         print(json.dumps(line))

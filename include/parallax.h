@@ -323,15 +323,20 @@ const char* parallax_status_string(int status);
  *
  *  - Arguments are those of parallax_decode without workspace and
  *    workspace_bytes; the same layouts, dtypes and errors apply.
- *  - A call whose workspace (parallax_decode_workspace_bytes for the same
- *    shape and num_splits) would exceed PARALLAX_NOALLOC_SCRATCH_BYTES is
- *    rejected with PARALLAX_ERR_SCRATCH_LIMIT before anything is launched.
- *    With D = 128 the array holds 1008 partitions for 2 query heads per kv
- *    head, 504 for 4 and 252 for 8 (the default is 2 per SM, 296 on a B200);
- *    pass a smaller num_splits for larger groups.
+ *  - Capacity: with D = 128 the array holds 1008 partitions for 2 query
+ *    heads per kv head, 504 for 4, 252 for 8 and 126 for 16 (twice as many
+ *    at D = 64). With num_splits = 0 the call takes the default count (one
+ *    partition per SM, 148 on a B200) capped at that capacity, so a default
+ *    call never fails for size. An explicit num_splits whose workspace
+ *    (parallax_decode_workspace_bytes for the same shape and count) exceeds
+ *    PARALLAX_NOALLOC_SCRATCH_BYTES is rejected with
+ *    PARALLAX_ERR_SCRATCH_LIMIT before anything is launched.
  *  - The first call on each device looks up the array's device address
- *    (cudaGetSymbolAddress) with that device current; make that first call
- *    before any stream capture.
+ *    (cudaGetSymbolAddress) with that device current and keeps it for the
+ *    life of the process; make that first call before any stream capture,
+ *    and do not use this entry point across a cudaDeviceReset (or any other
+ *    teardown of the device's primary context), which frees the array and
+ *    leaves the kept address stale.
  *  - Every call on a device shares the one array and leaves its contents
  *    behind; each call clears the status word at its start (a
  *    cudaMemsetAsync on `stream`). Calls that can overlap on the GPU (other

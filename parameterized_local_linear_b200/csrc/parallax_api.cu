@@ -6,6 +6,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstdlib>
@@ -59,18 +60,23 @@ struct Call {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// SM count of the current device, cached per device (host threads may call
+// concurrently: the cache entries are atomics).
 int current_sm_count(int* out) {
-  static int cache[256] = {0};
+  static std::atomic<int> cache[256];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return PARALLAX_ERR_CUDA;
-  if (dev >= 0 && dev < 256 && cache[dev] > 0) {
-    *out = cache[dev];
-    return PARALLAX_OK;
+  if (dev >= 0 && dev < 256) {
+    const int n = cache[dev].load(std::memory_order_relaxed);
+    if (n > 0) {
+      *out = n;
+      return PARALLAX_OK;
+    }
   }
   int n = 0;
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
     return PARALLAX_ERR_CUDA;
-  if (dev >= 0 && dev < 256) cache[dev] = n;
+  if (dev >= 0 && dev < 256) cache[dev].store(n, std::memory_order_relaxed);
   *out = n;
   return PARALLAX_OK;
 }
@@ -211,15 +217,18 @@ int encode_cache_map(CUtensorMap* map, const void* cache, int D, int Lmax, int H
 
 // ----------------------------------------------------------------- launch --
 
+// Raises the kernel's dynamic shared-memory limit once per device (the
+// attribute call is idempotent, so two threads racing here both succeed).
 template <typename Kernel>
-int set_smem_once(Kernel kernel, int bytes, int* done_dev) {
+int set_smem_once(Kernel kernel, int bytes, std::atomic<int>* done_dev) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return PARALLAX_ERR_CUDA;
-  if (dev >= 0 && dev < 256 && done_dev[dev] >= bytes) return PARALLAX_OK;
+  if (dev >= 0 && dev < 256 && done_dev[dev].load(std::memory_order_acquire) >= bytes)
+    return PARALLAX_OK;
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
       cudaSuccess)
     return PARALLAX_ERR_CUDA;
-  if (dev >= 0 && dev < 256) done_dev[dev] = bytes;
+  if (dev >= 0 && dev < 256) done_dev[dev].store(bytes, std::memory_order_release);
   return PARALLAX_OK;
 }
 
@@ -228,7 +237,7 @@ int launch_tc(const Call& c, const DecodeParams& prm, int P) {
   // probabilities as bf16 hi + lo: always with the probe, else for fp32 output
   constexpr bool kPsplit = PROBE || OUT_F32;
   auto kernel = parallax_tc_kernel<D, PROBE, OUT_F32, kPsplit>;
-  static int done[256] = {0};
+  static std::atomic<int> done[256];
   const TcSmemLayout L =
       tc_smem_layout(D, TcGeom<D>::kStageBytes, TcGeom<D>::kStages, prm.G, PROBE);
   int st = set_smem_once(kernel, L.total, done);
@@ -642,7 +651,7 @@ template <int D, bool OUT_F32, bool VARLEN>
 int launch_prefill(const void* q, const void* r, const void* k, const void* v,
                    const PrefillParams& prm, int grid_x, cudaStream_t stream) {
   auto kernel = parallax_prefill_kernel<D, OUT_F32, VARLEN>;
-  static int done[256] = {0};
+  static std::atomic<int> done[256];
   int st = set_smem_once(kernel, PfGeom<D>::kSmem, done);
   if (st != PARALLAX_OK) return st;
   CUtensorMap tq, tr, tk, tv;
@@ -832,7 +841,15 @@ extern "C" int parallax_decode_noalloc(const void* q, const void* r, const void*
   if ((st = validate(c)) != PARALLAX_OK) return st;
   int P = 0;
   if ((st = resolve_splits(num_splits, B, Hkv, Lmax, !tma_path(c), &P)) != PARALLAX_OK) return st;
-  if (workspace_bytes_for(Hq / Hkv, D, P) > kNoallocScratchBytes) return PARALLAX_ERR_SCRATCH_LIMIT;
+  // The default count is capped at what the array holds for this group and
+  // head size; an explicit count beyond it is an error.
+  const size_t per_split = workspace_bytes_for(Hq / Hkv, D, 1) - kWorkspaceHeaderBytes;
+  const int capacity = (int)std::min<size_t>(
+      PARALLAX_MAX_SPLITS, (kNoallocScratchBytes - kWorkspaceHeaderBytes) / per_split);
+  if (num_splits == 0) P = std::min(P, capacity);
+  if (P < 1 || workspace_bytes_for(Hq / Hkv, D, P) > kNoallocScratchBytes)
+    return PARALLAX_ERR_SCRATCH_LIMIT;
+  c.num_splits = P;
   // The array keeps the previous call's contents: the status word must start
   // at zero; the partial records are always written before they are read.
   if (cudaMemsetAsync(scratch, 0, kWorkspaceHeaderBytes, c.stream) != cudaSuccess)
