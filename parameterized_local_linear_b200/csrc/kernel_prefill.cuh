@@ -29,7 +29,11 @@
 //           with the weights the products apply. (One bf16 per weight is not
 //           enough: the value of key i is weighted by e_i (1 + s_i - b/l), so
 //           a weight's rounding error is multiplied by |s|, which for these
-//           probes reaches tens.) O is rescaled in TMEM only
+//           probes reaches tens.) With fp32 output the weights go in whole:
+//           e and e*s (fp32) are split into three bf16 terms hi + mid + lo,
+//           which sum to them exactly; hi and mid sit where P_hi and P_lo do,
+//           and the two lo tiles are A operands in shared memory (TMEM has no
+//           room left at D = 128). O is rescaled in TMEM only
 //           when the max grows by more than 2^8 (otherwise the stale max keeps
 //           every e <= 2^8); each thread of a row rescales one of O_A, O_C.
 // TMEM columns: S [0,64) T [64,128) P [128,256) (per key half, 64 columns:
@@ -62,14 +66,18 @@ struct PrefillParams {
   int debug_skip_first_k;   // testing hook: the producer never loads the first K tile
 };
 
-template <int D>
+template <int D, bool F32 = false>
 struct PfGeom {
   static constexpr int kH = D / 64;
   static constexpr int kQBytes = kH * kPfRows * 128;   // Q (or R) tile
   static constexpr int kKVBytes = kH * kPfKeys * 128;  // K (or V) tile
   static constexpr int kOffQ = 0, kOffR = kQBytes, kOffK = 2 * kQBytes;
   static constexpr int kOffV = kOffK + kPfStages * kKVBytes;
-  static constexpr int kOffRed = kOffV + kPfStages * kKVBytes;  // l, b of both key halves
+  // fp32 output: the lo terms of e and of e*s, one [128 rows][64 keys] bf16
+  // tile each, K-major with the 128-byte swizzle (the UMMA A-operand layout)
+  static constexpr int kP3Bytes = kPfRows * kPfKeys * 2;
+  static constexpr int kOffP3 = kOffV + kPfStages * kKVBytes;  // 1024-byte aligned
+  static constexpr int kOffRed = kOffP3 + (F32 ? 2 * kP3Bytes : 0);  // l, b of both key halves
   static constexpr int kOffBar = kOffRed + 4 * kPfRows * 4;
   static constexpr int kSmem = kOffBar + 256 + 1024;            // barriers, slots, alignment
   static constexpr uint32_t kColOA = 256, kColOC = 256 + D;
@@ -91,6 +99,19 @@ __device__ __forceinline__ float split_hi_lo(float x0, float x1, uint32_t& hi, u
   return y0 + y1;
 }
 
+// x0, x1 split into three bf16 terms hi + mid + lo that sum to them exactly
+// (each term rounds the remainder of the ones before to nearest; an fp32
+// value has 24 significant bits and each term takes 8). Packed as bf16x2
+// words (x0 in the low half). Returns x0 + x1.
+__device__ __forceinline__ float split3(float x0, float x1, uint32_t& hi, uint32_t& mid,
+                                        uint32_t& lo) {
+  hi = pack_bf16x2(x0, x1);
+  const float r0 = x0 - bf16_lo_to_float(hi), r1 = x1 - bf16_hi_to_float(hi);
+  mid = pack_bf16x2(r0, r1);
+  lo = pack_bf16x2(r0 - bf16_lo_to_float(mid), r1 - bf16_hi_to_float(mid));
+  return x0 + x1;
+}
+
 // VARLEN: the packed layout of parallax_varlen_func (q, r, out [total][Hq][D],
 // k, v [total][Hkv][D], sequence b in rows cu_seqlens[b] .. cu_seqlens[b+1]);
 // otherwise the dense [B][H][L][D] layout.
@@ -100,7 +121,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                             const __grid_constant__ CUtensorMap tmR,
                             const __grid_constant__ CUtensorMap tmK,
                             const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
-  using Geo = PfGeom<D>;
+  using Geo = PfGeom<D, OUT_F32>;
   constexpr uint32_t kIdescS = umma_idesc_bf16(kPfRows, kPfKeys, false);
   constexpr uint32_t kIdescPV = umma_idesc_bf16(kPfRows, D, true);
   const float kNegInf = __int_as_float(0xff800000u);
@@ -111,6 +132,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   uint8_t* const gbase = smem_raw + (base - raw);
   const uint32_t sQ = base + Geo::kOffQ, sR = base + Geo::kOffR;
   const uint32_t sK = base + Geo::kOffK, sV = base + Geo::kOffV;
+  const uint32_t sP3 = base + Geo::kOffP3;  // fp32 output: lo of e, then lo of e*s
   const uint32_t bar = base + Geo::kOffBar;
   const uint32_t bar_q = bar, k_full = bar + 8, k_empty = bar + 32, v_full = bar + 56,
                  v_empty = bar + 80;
@@ -284,6 +306,18 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                            acc);
             }
           }
+          if constexpr (OUT_F32) {  // the lo terms, A from shared memory: e -> O_A, e*s -> O_C
+#pragma unroll
+            for (int pm = 0; pm < 2; ++pm) {
+              const uint32_t dO = tmem + (pm == 0 ? Geo::kColOA : Geo::kColOC);
+              const uint32_t sA = sP3 + pm * Geo::kP3Bytes;
+#pragma unroll
+              for (int kk = 0; kk < kPfKeys / 16; ++kk)
+                umma_bf16(dO, umma_smem_desc(sA + 32 * kk, 16, 1024),
+                          umma_smem_desc(sVs + kk * 16 * 128, kPfKeys * 128, 1024), kIdescPV,
+                          true);
+            }
+          }
           umma_commit(o_done);
           umma_commit(v_empty + 8 * st);
         }
@@ -347,8 +381,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       }
       const float neg_m = -m_used;
       // e and e*s of this thread's 32 keys as exact bf16 hi + lo pairs, in the
-      // order of this half's P columns: P_hi | P_lo then PT_hi | PT_lo
+      // order of this half's P columns: P_hi | P_lo then PT_hi | PT_lo. With
+      // fp32 output: hi | mid in those columns and the lo terms in p3, pt3.
       uint32_t pp[32], pt[32];
+      uint32_t p3[OUT_F32 ? 16 : 1], pt3[OUT_F32 ? 16 : 1];
       uint32_t* const ph = pp;
       uint32_t* const pl = pp + 16;
       uint32_t* const th = pt;
@@ -358,11 +394,16 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       for (int u = 0; u < 16; ++u) {
         const float e0 = ex2_approx(fmaf(sv[2 * u], c, neg_m));
         const float e1 = ex2_approx(fmaf(sv[2 * u + 1], c, neg_m));
-        lt += split_hi_lo(e0, e1, ph[u], pl[u]);
-        // e*s from the rounded e: the weights P applies
-        const float es0 = round17(e0) * tv[2 * u];
-        const float es1 = round17(e1) * tv[2 * u + 1];
-        bt += split_hi_lo(es0, es1, th[u], tl[u]);
+        if constexpr (OUT_F32) {
+          lt += split3(e0, e1, ph[u], pl[u], p3[u]);
+          bt += split3(e0 * tv[2 * u], e1 * tv[2 * u + 1], th[u], tl[u], pt3[u]);
+        } else {
+          lt += split_hi_lo(e0, e1, ph[u], pl[u]);
+          // e*s from the rounded e: the weights P applies
+          const float es0 = round17(e0) * tv[2 * u];
+          const float es1 = round17(e1) * tv[2 * u + 1];
+          bt += split_hi_lo(es0, es1, th[u], tl[u]);
+        }
       }
       // the previous PV products must be done: P is single-buffered and O may be rescaled
       if (j > 0) {
@@ -388,6 +429,19 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       }
       l = l * alpha + lt;
       bsum = bsum * alpha + bt;
+      if constexpr (OUT_F32) {
+        // row r of the lo tiles: keys 32 half .. +31 are 16-byte chunks
+        // 4 half .. +3, each at chunk position (chunk ^ (r mod 8)) of the row
+        const uint32_t row = sP3 + (uint32_t)r * 128u, sw = (uint32_t)r & 7u;
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+          const uint32_t off = (((uint32_t)(4 * half + c4)) ^ sw) << 4;
+          st_shared_v4(row + off, p3[4 * c4], p3[4 * c4 + 1], p3[4 * c4 + 2], p3[4 * c4 + 3]);
+          st_shared_v4(row + Geo::kP3Bytes + off, pt3[4 * c4], pt3[4 * c4 + 1], pt3[4 * c4 + 2],
+                       pt3[4 * c4 + 3]);
+        }
+        fence_proxy_async_smem();  // the UMMAs read these tiles through the async proxy
+      }
       tmem_st32u(tP, pp);
       tmem_st32u(tP + 32, pt);
       tmem_wait_st();

@@ -652,7 +652,7 @@ int launch_prefill(const void* q, const void* r, const void* k, const void* v,
                    const PrefillParams& prm, int grid_x, cudaStream_t stream) {
   auto kernel = parallax_prefill_kernel<D, OUT_F32, VARLEN>;
   static std::atomic<int> done[256];
-  int st = set_smem_once(kernel, PfGeom<D>::kSmem, done);
+  int st = set_smem_once(kernel, PfGeom<D, OUT_F32>::kSmem, done);
   if (st != PARALLAX_OK) return st;
   CUtensorMap tq, tr, tk, tv;
   const void* src[4] = {q, r, k, v};
@@ -669,7 +669,7 @@ int launch_prefill(const void* q, const void* r, const void* k, const void* v,
   if (lin > 0x7fffffffLL) return PARALLAX_ERR_BAD_SHAPE;
   cfg.gridDim = dim3((unsigned)lin);
   cfg.blockDim = dim3(kPfThreads);
-  cfg.dynamicSmemBytes = PfGeom<D>::kSmem;
+  cfg.dynamicSmemBytes = PfGeom<D, OUT_F32>::kSmem;
   cfg.stream = stream;
   return cudaLaunchKernelEx(&cfg, kernel, tq, tr, tk, tv, prm) == cudaSuccess ? PARALLAX_OK
                                                                               : PARALLAX_ERR_CUDA;

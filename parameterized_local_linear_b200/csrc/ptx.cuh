@@ -115,6 +115,13 @@ __device__ __forceinline__ uint64_t l2_policy_evict_first() {
 
 // Order this thread's generic-proxy shared-memory writes before later
 // async-proxy (TMA) writes to the same bytes.
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }

@@ -15,7 +15,7 @@ pytestmark = pytest.mark.gpu
 TOL = {torch.bfloat16: 2e-2, torch.float32: 1e-4}
 
 
-def make(lens, Hq, Hkv, D, seed, r_scale=0.5):
+def make(lens, Hq, Hkv, D, seed, r_scale=1.0):
     g = torch.Generator(device="cuda").manual_seed(seed)
     total = int(sum(lens))
     rnd = lambda H, s=1.0: (torch.randn(total, H, D, device="cuda", generator=g) * s).to(torch.bfloat16)
@@ -38,11 +38,12 @@ def scaled_error(got, ref):
     return float(np.max(np.abs(g - ref) / np.maximum(1.0, np.abs(ref))))
 
 
+@pytest.mark.parametrize("r_scale", [0.5, 1.0, 2.0])
 @pytest.mark.parametrize("D", [64, 128])
 @pytest.mark.parametrize("Hq,Hkv", [(2, 2), (4, 2)])
-def test_varlen_matches_oracle(D, Hq, Hkv):
+def test_varlen_matches_oracle(D, Hq, Hkv, r_scale):
     lens = [1, 130, 64, 0, 257, 5, 128]
-    q, r, k, v, cu = make(lens, Hq, Hkv, D, seed=400 + D + Hq)
+    q, r, k, v, cu = make(lens, Hq, Hkv, D, seed=400 + D + Hq, r_scale=r_scale)
     scale = D ** -0.5
     ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
     for causal in (True, False):
@@ -51,7 +52,7 @@ def test_varlen_matches_oracle(D, Hq, Hkv):
             got = binding.parallax_varlen_prefill(q, r, k, v, cu, max(lens), scale=scale,
                                                   causal=causal, out_dtype=out_dtype, workspace=ws)
             err = scaled_error(got, want)
-            assert err <= TOL[out_dtype], (D, Hq, Hkv, causal, out_dtype, err)
+            assert err <= TOL[out_dtype], (D, Hq, Hkv, r_scale, causal, out_dtype, err)
     torch.cuda.synchronize()
     assert int(ws[:4].view(torch.int32).item()) == 0
 
