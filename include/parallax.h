@@ -202,7 +202,8 @@ int parallax_decode_phase(int phase, int probe, const void* q, const void* r,
  * Decode over a paged KV cache: the pages' decode (parallax-kernel 0.1.0
  * README, "Decoding (CuTeDSL)") with its (B, kv_len, H, D) cache cut into
  * fixed-size pages, the layout serving engines keep their caches in.
- *  - k_pages, v_pages [num_pages][page_size][Hkv][D] bf16 (a pool of pages);
+ *  - k_pages, v_pages [num_pages][page_size][Hkv][D] (a pool of pages), bf16
+ *    or fp32 (in_dtype, which q and r share);
  *    block_table [B][max_pages_per_seq] int32: key i of sequence b is slot
  *    i % page_size of page block_table[b][i / page_size]. Only the entries a
  *    sequence's length reaches are read.
@@ -212,16 +213,18 @@ int parallax_decode_phase(int phase, int probe, const void* q, const void* r,
  *  - A page id outside [0, num_pages) is not read: its keys are left out and
  *    PARALLAX_DEVICE_STATUS_SEQLEN_CLAMPED is set.
  *  - probe != 0: the Parallax output (r required); probe == 0: R = 0 softmax.
- *  - bf16 inputs; any query-head group (groups of more than 4 query heads per
- *    kv head with the probe, or 8 without, go through the generic kernel).
+ *  - bf16 or fp32 inputs (in_dtype); any query-head group. bf16 pools with
+ *    up to 4 query heads per kv head with the probe (8 without) run on the
+ *    TMA kernel; fp32 pools and larger groups on the generic kernel, which
+ *    resolves the pages the same way.
  *  - Workspace: parallax_decode_workspace_bytes(B, Hq, Hkv, D,
  *    max_pages_per_seq * page_size, num_splits). Other rules as parallax_decode.
  */
 int parallax_decode_paged(const void* q, const void* r, const void* k_pages, const void* v_pages,
                           const int32_t* block_table, const int32_t* cache_seqlens, void* out,
                           int B, int Hq, int Hkv, int D, float scale, void* stream, int num_pages,
-                          int page_size, int max_pages_per_seq, int probe, int out_dtype,
-                          int num_splits, void* workspace, size_t workspace_bytes);
+                          int page_size, int max_pages_per_seq, int probe, int in_dtype,
+                          int out_dtype, int num_splits, void* workspace, size_t workspace_bytes);
 
 /*
  * Block-sparse decode: parallax-kernel 0.1.0 README (opening section) notes
@@ -235,7 +238,8 @@ int parallax_decode_paged(const void* q, const void* r, const void* k_pages, con
  *  - A block id outside [0, ceil(Lmax / 64)) or a count outside [0,
  *    max_blocks] is clamped away and sets PARALLAX_DEVICE_STATUS_SEQLEN_CLAMPED.
  *  - A block listed twice is attended twice (its keys count twice).
- *  - bf16 inputs; any query-head group, as parallax_decode_paged.
+ *  - bf16 or fp32 inputs (in_dtype); any query-head group, as
+ *    parallax_decode_paged.
  *  - Workspace: parallax_decode_workspace_bytes(B, Hq, Hkv, D, 64 * max_blocks,
  *    num_splits). Other rules as parallax_decode.
  */
@@ -243,8 +247,9 @@ int parallax_decode_block_sparse(const void* q, const void* r, const void* k_cac
                                  const void* v_cache, const int32_t* cache_seqlens,
                                  const int32_t* block_ids, const int32_t* num_blocks, void* out,
                                  int B, int Hq, int Hkv, int D, float scale, void* stream, int Lmax,
-                                 int kv_layout, int max_blocks, int probe, int out_dtype,
-                                 int num_splits, void* workspace, size_t workspace_bytes);
+                                 int kv_layout, int max_blocks, int probe, int in_dtype,
+                                 int out_dtype, int num_splits, void* workspace,
+                                 size_t workspace_bytes);
 
 /*
  * The training-shape (prefill) forward: parallax-kernel 0.1.0 README,

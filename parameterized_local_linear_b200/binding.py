@@ -43,9 +43,10 @@ def load_library():
     lib.parallax_softmax_decode.argtypes = [vp, vp, vp, vp, vp] + decode_tail
     lib.parallax_decode_phase.argtypes = [i, i, vp, vp, vp, vp, vp, vp] + decode_tail
     lib.parallax_decode_ex.argtypes = [vp, vp, vp, vp, vp, vp] + decode_tail + [i, i, i, i]
-    lib.parallax_decode_paged.argtypes = [vp] * 7 + [i, i, i, i, f, vp, i, i, i, i, i, i, vp, sz]
+    lib.parallax_decode_paged.argtypes = [vp] * 7 + [i, i, i, i, f, vp, i, i, i, i, i, i, i, vp,
+                                                     sz]
     lib.parallax_decode_block_sparse.argtypes = ([vp] * 8 + [i, i, i, i, f, vp, i, i, i, i, i, i,
-                                                             vp, sz])
+                                                             i, vp, sz])
     lib.parallax_decode_workspace_bytes.argtypes = [i, i, i, i, i, i]
     lib.parallax_decode_workspace_bytes.restype = sz
     lib.parallax_choose_splits.argtypes = [i, i, i, i]
@@ -320,11 +321,17 @@ def parallax_decode_paged(q, r, k_pages, v_pages, block_table, cache_seqlens=Non
                           workspace: Optional[Workspace] = None, num_splits: int = 0,
                           probe: bool = True, stream=None):
     """Decode over a paged cache: k_pages, v_pages [num_pages, page_size, Hkv, D]
-    bf16, block_table int32 [B, max_pages_per_seq] (page ids per sequence),
-    cache_seqlens int32 [B] or None (every sequence fills its table)."""
+    bf16 or fp32 (q's dtype), block_table int32 [B, max_pages_per_seq] (page
+    ids per sequence), cache_seqlens int32 [B] or None (every sequence fills
+    its table)."""
     for name, t in (("q", q), ("k_pages", k_pages), ("v_pages", v_pages)):
-        if not t.is_cuda or not t.is_contiguous() or t.dtype != torch.bfloat16:
-            raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor")
+        if not t.is_cuda or not t.is_contiguous() or t.dtype not in _DTYPE_CODE:
+            raise ValueError(f"{name} must be a contiguous bf16 or fp32 CUDA tensor")
+        if t.dtype != q.dtype:
+            raise ValueError("q, r, k_pages, v_pages must share one dtype")
+    if probe and (r is None or r.shape != q.shape or r.dtype != q.dtype or not r.is_cuda
+                  or not r.is_contiguous()):
+        raise ValueError("r must be a contiguous CUDA tensor shaped like q")
     if q.dim() != 3 or k_pages.dim() != 4 or v_pages.shape != k_pages.shape:
         raise ValueError("expected q [B,Hq,D] and k_pages, v_pages [num_pages,page_size,Hkv,D]")
     B, Hq, D = q.shape
@@ -346,8 +353,8 @@ def parallax_decode_paged(q, r, k_pages, v_pages, block_table, cache_seqlens=Non
     rc = load_library().parallax_decode_paged(
         q.data_ptr(), _ptr(r) if probe else None, k_pages.data_ptr(), v_pages.data_ptr(),
         block_table.data_ptr(), _ptr(cache_seqlens), out.data_ptr(), B, Hq, Hkv, D, float(scale),
-        _stream(stream), num_pages, page_size, max_pages, int(bool(probe)), _DTYPE_CODE[out.dtype],
-        int(num_splits), workspace.ptr(), workspace.nbytes)
+        _stream(stream), num_pages, page_size, max_pages, int(bool(probe)), _DTYPE_CODE[q.dtype],
+        _DTYPE_CODE[out.dtype], int(num_splits), workspace.ptr(), workspace.nbytes)
     _check(rc, "parallax_decode_paged")
     return out
 
@@ -358,8 +365,12 @@ def parallax_decode_block_sparse(q, r, k_cache, v_cache, block_ids, num_blocks,
                                  num_splits: int = 0, probe: bool = True, kv_layout: str = "bhsd",
                                  stream=None):
     """Decode over the listed 64-key blocks of each sequence: block_ids int32
-    [B, max_blocks] (first num_blocks[b] used), num_blocks int32 [B]."""
+    [B, max_blocks] (first num_blocks[b] used), num_blocks int32 [B]; bf16 or
+    fp32 inputs."""
     B, Hq, Hkv, D, Lmax = _shapes(q, k_cache, v_cache, cache_seqlens, kv_layout)
+    if probe and (r is None or r.shape != q.shape or r.dtype != q.dtype or not r.is_cuda
+                  or not r.is_contiguous()):
+        raise ValueError("r must be a contiguous CUDA tensor shaped like q")
     _check_int32("block_ids", block_ids, 2)
     _check_int32("num_blocks", num_blocks, 1)
     if block_ids.shape[0] != B or num_blocks.shape != (B,):
@@ -375,8 +386,8 @@ def parallax_decode_block_sparse(q, r, k_cache, v_cache, block_ids, num_blocks,
         q.data_ptr(), _ptr(r) if probe else None, k_cache.data_ptr(), v_cache.data_ptr(),
         _ptr(cache_seqlens), block_ids.data_ptr(), num_blocks.data_ptr(), out.data_ptr(), B, Hq,
         Hkv, D, float(scale), _stream(stream), Lmax, KV_LAYOUTS[kv_layout], max_blocks,
-        int(bool(probe)), _DTYPE_CODE[out.dtype], int(num_splits), workspace.ptr(),
-        workspace.nbytes)
+        int(bool(probe)), _DTYPE_CODE[q.dtype], _DTYPE_CODE[out.dtype], int(num_splits),
+        workspace.ptr(), workspace.nbytes)
     _check(rc, "parallax_decode_block_sparse")
     return out
 

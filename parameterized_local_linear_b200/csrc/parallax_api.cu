@@ -153,7 +153,6 @@ int validate(const Call& c) {
       return PARALLAX_ERR_BAD_SHAPE;
     if (c.kv_mode == kKvBlockSparse && (long long)c.table_stride * kTileKeys > 0x7fffffffLL)
       return PARALLAX_ERR_BAD_SHAPE;
-    if (c.in_dtype != PARALLAX_DTYPE_BF16) return PARALLAX_ERR_UNSUPPORTED_DTYPE;  // bf16 pools
   }
   if (c.probe && !c.r) return PARALLAX_ERR_NULL_POINTER;
   if (!shape_ok(c.B, c.Hq, c.Hkv, c.D, c.Lmax)) return PARALLAX_ERR_BAD_SHAPE;
@@ -485,14 +484,14 @@ int parallax_decode_ex(const void* q, const void* r, const void* k_cache, const 
 int parallax_decode_paged(const void* q, const void* r, const void* k_pages, const void* v_pages,
                           const int32_t* block_table, const int32_t* cache_seqlens, void* out,
                           int B, int Hq, int Hkv, int D, float scale, void* stream, int num_pages,
-                          int page_size, int max_pages_per_seq, int probe, int out_dtype,
-                          int num_splits, void* workspace, size_t workspace_bytes) {
+                          int page_size, int max_pages_per_seq, int probe, int in_dtype,
+                          int out_dtype, int num_splits, void* workspace, size_t workspace_bytes) {
   if (page_size < 1 || max_pages_per_seq < 1) return PARALLAX_ERR_BAD_SHAPE;
   const long long lmax = (long long)page_size * max_pages_per_seq;
   if (lmax > 0x7fffffffLL) return PARALLAX_ERR_BAD_SHAPE;
   Call c = make_call(3, probe != 0, q, r, k_pages, v_pages, cache_seqlens, out, B, Hq, Hkv, D,
-                     scale, stream, (int)lmax, PARALLAX_DTYPE_BF16, out_dtype, num_splits,
-                     workspace, workspace_bytes);
+                     scale, stream, (int)lmax, in_dtype, out_dtype, num_splits, workspace,
+                     workspace_bytes);
   c.kv_mode = kKvPaged;
   c.table = block_table;
   c.table_stride = max_pages_per_seq;
@@ -505,10 +504,11 @@ int parallax_decode_block_sparse(const void* q, const void* r, const void* k_cac
                                  const void* v_cache, const int32_t* cache_seqlens,
                                  const int32_t* block_ids, const int32_t* num_blocks, void* out,
                                  int B, int Hq, int Hkv, int D, float scale, void* stream, int Lmax,
-                                 int kv_layout, int max_blocks, int probe, int out_dtype,
-                                 int num_splits, void* workspace, size_t workspace_bytes) {
+                                 int kv_layout, int max_blocks, int probe, int in_dtype,
+                                 int out_dtype, int num_splits, void* workspace,
+                                 size_t workspace_bytes) {
   Call c = make_call(3, probe != 0, q, r, k_cache, v_cache, cache_seqlens, out, B, Hq, Hkv, D,
-                     scale, stream, Lmax, PARALLAX_DTYPE_BF16, out_dtype, num_splits, workspace,
+                     scale, stream, Lmax, in_dtype, out_dtype, num_splits, workspace,
                      workspace_bytes);
   c.kv_layout = kv_layout;
   c.kv_mode = kKvBlockSparse;

@@ -3,8 +3,8 @@ reading 64-key tiles through a page table or a per-sequence block list)
 against the fp64 oracle, which gathers the same keys into a dense cache:
 ragged lengths that end inside a page or block, a shuffled page pool, unsorted
 and repeated block lists, empty selections, both cache layouts, GQA groups,
-Parallax and R = 0, bf16 and fp32 outputs, several split counts, and the
-device-side handling of ids outside the pool or the cache."""
+Parallax and R = 0, bf16 and fp32 inputs and outputs, several split counts,
+and the device-side handling of ids outside the pool or the cache."""
 import numpy as np
 import pytest
 import torch
@@ -28,13 +28,13 @@ def status_bits(ws):
     return bits
 
 
-def paged_case(seed, B, Hq, Hkv, D, page_size, max_pages, lens, spare=5):
+def paged_case(seed, B, Hq, Hkv, D, page_size, max_pages, lens, spare=5, dtype=torch.bfloat16):
     g = torch.Generator(device="cuda").manual_seed(seed)
     num_pages = B * max_pages + spare
-    q = torch.randn(B, Hq, D, device="cuda", generator=g).to(torch.bfloat16)
-    r = (torch.randn(B, Hq, D, device="cuda", generator=g) * 0.5).to(torch.bfloat16)
-    kp = torch.randn(num_pages, page_size, Hkv, D, device="cuda", generator=g).to(torch.bfloat16)
-    vp = torch.randn(num_pages, page_size, Hkv, D, device="cuda", generator=g).to(torch.bfloat16)
+    q = torch.randn(B, Hq, D, device="cuda", generator=g).to(dtype)
+    r = (torch.randn(B, Hq, D, device="cuda", generator=g) * 0.5).to(dtype)
+    kp = torch.randn(num_pages, page_size, Hkv, D, device="cuda", generator=g).to(dtype)
+    vp = torch.randn(num_pages, page_size, Hkv, D, device="cuda", generator=g).to(dtype)
     perm = torch.randperm(num_pages, generator=torch.Generator().manual_seed(seed))
     table = perm[:B * max_pages].reshape(B, max_pages).to(torch.int32).cuda()
     n = torch.tensor(lens, dtype=torch.int32, device="cuda")
@@ -63,6 +63,27 @@ def test_paged_matches_oracle(D, Hq, Hkv, page_size):
                 assert status_bits(ws) == 0
 
 
+@pytest.mark.parametrize("D,Hq,Hkv", [(128, 16, 8), (64, 8, 8), (128, 16, 2)])
+@pytest.mark.parametrize("page_size", [64, 192])
+def test_paged_f32_pool_matches_oracle(D, Hq, Hkv, page_size):
+    """fp32 pools (q, r, pages all fp32) on the generic kernel, lengths that
+    end inside a page, both output dtypes, Parallax and R = 0."""
+    max_pages = (2048 + page_size - 1) // page_size
+    lens = [1, 333, 2048]
+    q, r, kp, vp, table, n = paged_case(530 + D + page_size, 3, Hq, Hkv, D, page_size,
+                                        max_pages, lens, dtype=torch.float32)
+    for probe in (True, False):
+        want = oracle.parallax_decode_paged(q, r, kp, vp, table, n, D ** -0.5, probe=probe)
+        for out_dtype in (torch.bfloat16, torch.float32):
+            for splits in (0, 3):
+                ws = binding.Workspace(3, Hq, Hkv, D, max_pages * page_size, splits)
+                got = binding.parallax_decode_paged(q, r, kp, vp, table, n, out_dtype=out_dtype,
+                                                    workspace=ws, num_splits=splits, probe=probe)
+                err = scaled_error(got, want)
+                assert err <= TOL[out_dtype], (probe, out_dtype, splits, err)
+                assert status_bits(ws) == 0
+
+
 def test_paged_without_lengths_and_bad_page():
     q, r, kp, vp, table, n = paged_case(520, 2, 16, 8, 128, 64, 10, [640, 640])
     want = oracle.parallax_decode_paged(q, r, kp, vp, table, None, 128 ** -0.5)
@@ -80,13 +101,13 @@ def test_paged_without_lengths_and_bad_page():
     assert scaled_error(got[0], want[0]) <= 1e-4  # the other sequence is untouched
 
 
-def sparse_case(seed, B, Hq, Hkv, D, Lmax, lens, layout):
+def sparse_case(seed, B, Hq, Hkv, D, Lmax, lens, layout, dtype=torch.bfloat16):
     g = torch.Generator(device="cuda").manual_seed(seed)
-    q = torch.randn(B, Hq, D, device="cuda", generator=g).to(torch.bfloat16)
-    r = (torch.randn(B, Hq, D, device="cuda", generator=g) * 0.5).to(torch.bfloat16)
+    q = torch.randn(B, Hq, D, device="cuda", generator=g).to(dtype)
+    r = (torch.randn(B, Hq, D, device="cuda", generator=g) * 0.5).to(dtype)
     shape = (B, Hkv, Lmax, D) if layout == "bhsd" else (B, Lmax, Hkv, D)
-    k = torch.randn(*shape, device="cuda", generator=g).to(torch.bfloat16)
-    v = torch.randn(*shape, device="cuda", generator=g).to(torch.bfloat16)
+    k = torch.randn(*shape, device="cuda", generator=g).to(dtype)
+    v = torch.randn(*shape, device="cuda", generator=g).to(dtype)
     n = torch.tensor(lens, dtype=torch.int32, device="cuda")
     return q, r, k, v, n
 
@@ -120,6 +141,38 @@ def test_block_sparse_matches_oracle(layout, D, Hq, Hkv):
                 err = scaled_error(got, want)
                 assert err <= TOL[out_dtype], (probe, out_dtype, splits, err)
                 assert torch.all(got[3] == 0)  # no block listed: zero output
+                assert status_bits(ws) == 0
+
+
+@pytest.mark.parametrize("layout", ["bhsd", "bshd"])
+@pytest.mark.parametrize("D,Hq,Hkv", [(64, 8, 4), (128, 16, 8)])
+def test_block_sparse_f32_matches_oracle(layout, D, Hq, Hkv):
+    """fp32 caches on the generic kernel: unsorted, repeated and
+    past-the-length blocks, an empty list, both layouts and output dtypes."""
+    B, Lmax, nblk = 4, 2048, 32
+    lens = [2048, 700, 37, 2048]
+    q, r, k, v, n = sparse_case(620 + D, B, Hq, Hkv, D, Lmax, lens, layout, dtype=torch.float32)
+    rng = np.random.default_rng(621)
+    ids = np.zeros((B, 12), dtype=np.int32)
+    cnt = np.array([12, 8, 3, 0], dtype=np.int32)
+    ids[0] = rng.choice(nblk, 12, replace=False)
+    ids[1, :8] = np.sort(rng.choice(nblk, 8, replace=False))
+    ids[2, :3] = [0, 0, 5]
+    bid, bcnt = torch.from_numpy(ids).cuda(), torch.from_numpy(cnt).cuda()
+    k_o = k if layout == "bhsd" else k.transpose(1, 2)
+    v_o = v if layout == "bhsd" else v.transpose(1, 2)
+    for probe in (True, False):
+        want = oracle.parallax_decode_block_sparse(q, r, k_o, v_o, ids, cnt, n, D ** -0.5,
+                                                   probe=probe)
+        for out_dtype in (torch.bfloat16, torch.float32):
+            for splits in (0, 4):
+                ws = binding.Workspace(B, Hq, Hkv, D, 64 * 12, splits)
+                got = binding.parallax_decode_block_sparse(
+                    q, r, k, v, bid, bcnt, n, out_dtype=out_dtype, workspace=ws,
+                    num_splits=splits, probe=probe, kv_layout=layout)
+                err = scaled_error(got, want)
+                assert err <= TOL[out_dtype], (probe, out_dtype, splits, err)
+                assert torch.all(got[3] == 0)
                 assert status_bits(ws) == 0
 
 
