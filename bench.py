@@ -46,9 +46,14 @@ FALLBACK_BF16_TFLOPS = 1590.0
 PREFILL_DEFAULT_SHAPE = "4,16,8,4096,128"
 DEFAULT_STEPS = {"tiny": 20000, "qwen": 100000, "large": 200, "long": 200, "ragged": 200}
 DEFAULT_WARMUP = {"tiny": 2000, "qwen": 5000, "large": 5, "long": 5, "ragged": 5}
-# the sources that decide what the split-KV kernel does (hashed against the ncu summary)
-MAIN_KERNEL_SRCS = [os.path.join(ROOT, "parameterized_local_linear_b200", "csrc", f)
-                    for f in ("kernel_tc.cuh", "partition.cuh", "common.cuh", "ptx.cuh")]
+# the sources that decide what each decode kernel does (hashed against its ncu summary)
+_CSRC = os.path.join(ROOT, "parameterized_local_linear_b200", "csrc")
+KERNEL_SRCS = {
+    "tc": [os.path.join(_CSRC, f) for f in ("kernel_tc.cuh", "partition.cuh", "common.cuh",
+                                            "ptx.cuh")],
+    "cluster": [os.path.join(_CSRC, f) for f in ("kernel_cluster.cuh", "kernel_tc.cuh",
+                                                 "common.cuh", "ptx.cuh")],
+}
 
 
 def parse_args():
@@ -131,34 +136,37 @@ def measured_bf16_peak():
         return FALLBACK_BF16_TFLOPS, "fallback"
 
 
-# ncu summaries whose traffic line the bench reports, per workload: (file,
-# batch rows the capture ran). A capture on fewer rows than the workload is
-# scaled by the rows processed (every row of these workloads has the same
-# length, so the split-KV kernel's traffic grows in proportion).
-PROFILE_FOR = {"qwen": ("parallax_tc_kernel_qwen.md", 1),
-               "large": ("parallax_tc_kernel_large_B64.md", 64)}
+# ncu summaries whose traffic line the bench reports, per (workload, kernel):
+# (file, batch rows the capture ran). A capture on fewer rows than the
+# workload is scaled by the rows processed (every row of these workloads has
+# the same length, so the kernel's traffic grows in proportion).
+PROFILE_FOR = {("qwen", "cluster"): ("parallax_cluster_kernel_qwen.md", 1),
+               ("large", "tc"): ("parallax_tc_kernel_large_B64.md", 64)}
 
 
-def profiled_traffic(w):
-    """Per-launch DRAM traffic (read + write) of the split-KV kernel from the
-    committed ncu summary of this workload, if it was taken on the current
+def source_hash(kernel):
+    h = hashlib.sha256()
+    for f in KERNEL_SRCS[kernel]:
+        h.update(open(f, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(w, kernel):
+    """Per-launch DRAM traffic (read + write) of the workload's dominant
+    kernel from its committed ncu summary, if that was taken on the current
     kernel source; scaled to the workload's batch when captured on fewer
     rows. None otherwise."""
     name = w.name.split("-")[0]
-    if name not in PROFILE_FOR or w.name != name:
+    if (name, kernel) not in PROFILE_FOR or w.name != name:
         return None
-    fname, rows = PROFILE_FOR[name]
+    fname, rows = PROFILE_FOR[(name, kernel)]
     try:
         text = open(os.path.join(ROOT, "profiles", fname)).read()
     except OSError:
         return None
-    h = hashlib.sha256()
-    for f in MAIN_KERNEL_SRCS:
-        h.update(open(f, "rb").read())
-    src_hash = h.hexdigest()[:16]
     m_hash = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
     m_traffic = re.search(r"traffic_bytes_per_launch:\s*([0-9]+)", text)
-    if not m_hash or not m_traffic or m_hash.group(1) != src_hash:
+    if not m_hash or not m_traffic or m_hash.group(1) != source_hash(kernel):
         return None
     return int(m_traffic.group(1)) * w.B // rows
 
@@ -859,6 +867,12 @@ class DecodeRig:
         self.bufs = [x] + [{k: (v.clone() if torch.is_tensor(v) else v) for k, v in x.items()}
                            for _ in range(self.nbuf - 1)]
         self.out = torch.empty((w.B, w.Hq, w.D), device=dev, dtype=out_dtype)
+        # num_splits = 0: the library's own schedule (a cluster per item for few
+        # items, else split-KV partitions + merge); > 0 forces that many partitions
+        self.num_splits = num_splits
+        self.plan = (binding.parallax_decode_plan(w.B, w.Hq, w.Hkv, w.D, w.Lmax, w.dtype,
+                                                  out_dtype) if num_splits == 0
+                     else {"grid_ctas": num_splits, "cluster_ctas": 0})
         self.P = (num_splits if num_splits > 0 else
                   binding.parallax_default_splits(w.B, w.Hq, w.Hkv, w.Lmax, w.dtype))
         self.ws = binding.Workspace(w.B, w.Hq, w.Hkv, w.D, w.Lmax, self.P, device=dev)
@@ -869,12 +883,12 @@ class DecodeRig:
         bd = self.binding
         if probe:
             bd.parallax_decode(b["q"], b["r"], b["k"], b["v"], b["seqlens"], scale=b["scale"],
-                               out=self.out, num_splits=self.P, workspace=self.ws,
+                               out=self.out, num_splits=self.num_splits, workspace=self.ws,
                                stream=self.stream)
         else:
             bd.parallax_softmax_decode(b["q"], b["k"], b["v"], b["seqlens"], scale=b["scale"],
-                                       out=self.out, num_splits=self.P, workspace=self.ws,
-                                       stream=self.stream)
+                                       out=self.out, num_splits=self.num_splits,
+                                       workspace=self.ws, stream=self.stream)
 
     def _make_runner(self, probe):
         """run(k) enqueues exactly k steps. Graph-replayed workloads replay
@@ -1018,7 +1032,7 @@ def qwen_companion(dev, stream, dist):
     for _ in range(20):
         per_trial.append(gated_region(stream, lambda: run(n_trial), host * n_trial) / n_trial)
     per_trial.sort()
-    out = {"workload": workload_desc(w), "num_splits": rig.P, "l2": rig.l2_note,
+    out = {"workload": workload_desc(w), "plan": rig.plan, "l2": rig.l2_note,
            "us_per_step_same_blocks": dist.max(t_p) * 1e6,
            "softmax_r0_us_per_step": dist.max(t_s) * 1e6,
            "parallax_over_softmax_latency": t_p / t_s,
@@ -1097,11 +1111,18 @@ def main():
     if rc != 0:
         raise SystemExit(f"device status after timing: {binding.parallax_status_string(rc)}")
 
-    # ---- per-launch duration of the split-KV kernel (phase 1 only), live ----
-    # Back-to-back phase-1 launches (each waits for the previous one's end, so
-    # the period is one launch's duration). Launch-bound sizes replay them from
-    # a CUDA graph; large ones are timed with events around each launch.
+    # ---- per-launch duration of the dominant kernel, live ----
+    # The split-KV kernel alone (phase 1) on the partition path; on the
+    # cluster path the step is that one kernel. Back-to-back launches (each
+    # waits for the previous one's end, so the period is one launch's
+    # duration). Launch-bound sizes replay them from a CUDA graph; large ones
+    # are timed with events around each launch.
+    cluster = rig.plan["cluster_ctas"] > 0
+
     def phase1(b):
+        if cluster:
+            step(b)
+            return
         binding.parallax_decode_phase(1, True, b["q"], b["r"], b["k"], b["v"], b["seqlens"],
                                       out, ws, scale=b["scale"], num_splits=P, stream=stream)
 
@@ -1265,7 +1286,8 @@ def main():
         "data": "synthetic",
         "config": {"workload": workload_desc(w), "global_batch": w.B * N, "seq_len": w.Lmax,
                    "parallelism": f"replicas x{N}" if N > 1 else "single GPU",
-                   "num_splits": P, "l2": rig.l2_note, "cuda_graphs": use_graphs,
+                   "num_splits": args.num_splits, "plan": rig.plan, "l2": rig.l2_note,
+                   "cuda_graphs": use_graphs,
                    "out_dtype": args.out_dtype,
                    "timing": "CUDA events around exactly K steps, enqueued behind a sleep "
                              "kernel so that no host launch gap is timed"},
@@ -1285,10 +1307,13 @@ def main():
         "e2e": {"value": N * k_e2e * step_kv / t_e2e / 1e9, "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "us_per_step": t_e2e / k_e2e * 1e6, "transfer": transfer},
-        "gpu_launches": 2 * args.steps,  # split-KV + merge per step, in the timed region
+        # split-KV + merge per step, or the one cluster kernel, in the timed region
+        "gpu_launches": (1 if cluster else 2) * args.steps,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": achieved / hbm_peak, "traffic": profiled_traffic(w),
-                     "kernel": "parallax_tc_kernel (split-KV)", "peak_source": peak_src,
+                     "frac": achieved / hbm_peak,
+                     "traffic": profiled_traffic(w, "cluster" if cluster else "tc"),
+                     "kernel": ("parallax_cluster_kernel (the whole step)" if cluster
+                                else "parallax_tc_kernel (split-KV)"), "peak_source": peak_src,
                      "kernel_us": main_s * 1e6, "launches_timed": main_launches,
                      "algorithmic_bytes_per_launch": main_bytes},
         "cpu_baseline": cpu,

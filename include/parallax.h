@@ -199,6 +199,25 @@ int parallax_decode_phase(int phase, int probe, const void* q, const void* r,
                           void* workspace, size_t workspace_bytes);
 
 /*
+ * How a decode call with num_splits = 0 runs these shapes on the current
+ * device (contiguous cache, no window). Two schedules exist:
+ *  - split-KV + merge: *grid_ctas partitions of the flattened key range (one
+ *    CTA each), partial records in the workspace, then the merge kernel;
+ *    *cluster_ctas = 0.
+ *  - one thread-block cluster per (batch row, kv head) item, for few items
+ *    (B * Hkv at most half the SM count) on the TMA kernel's inputs: the
+ *    item's 64-key tiles are dealt round-robin to *cluster_ctas CTAs (2 to
+ *    16, the most that leave every cluster resident at once), which combine
+ *    their (m, l, b, A, C) through distributed shared memory; no merge
+ *    kernel and no partial records; *grid_ctas = B * Hkv * *cluster_ctas.
+ * The results of the two agree within the decode tolerances (the sums are
+ * grouped differently); each is deterministic. An explicit num_splits > 0
+ * always takes the first. Returns PARALLAX_OK or an argument error.
+ */
+int parallax_decode_plan(int B, int Hq, int Hkv, int D, int Lmax, int in_dtype, int out_dtype,
+                         int probe, int* grid_ctas, int* cluster_ctas);
+
+/*
  * Decode over a paged KV cache: the pages' decode (parallax-kernel 0.1.0
  * README, "Decoding (CuTeDSL)") with its (B, kv_len, H, D) cache cut into
  * fixed-size pages, the layout serving engines keep their caches in.

@@ -128,6 +128,19 @@ def parallax_default_splits(B: int, Hq: int, Hkv: int, Lmax: int, dtype=torch.bf
     return n
 
 
+def parallax_decode_plan(B: int, Hq: int, Hkv: int, D: int, Lmax: int, dtype=torch.bfloat16,
+                         out_dtype=torch.bfloat16, probe: bool = True) -> dict:
+    """How a decode call with num_splits=0 runs these shapes: the grid size and
+    the CTAs per cluster (0: split-KV partitions + merge kernel)."""
+    fn = load_library().parallax_decode_plan
+    fn.argtypes = [ctypes.c_int] * 8 + [ctypes.POINTER(ctypes.c_int)] * 2
+    fn.restype = ctypes.c_int
+    grid, cl = ctypes.c_int(0), ctypes.c_int(0)
+    _check(fn(B, Hq, Hkv, D, Lmax, _DTYPE_CODE[dtype], _DTYPE_CODE[out_dtype], int(bool(probe)),
+              ctypes.byref(grid), ctypes.byref(cl)), "parallax_decode_plan")
+    return {"grid_ctas": grid.value, "cluster_ctas": cl.value}
+
+
 def parallax_decode_workspace_bytes(B: int, Hq: int, Hkv: int, D: int, Lmax: int,
                                     num_splits: int = 0) -> int:
     n = load_library().parallax_decode_workspace_bytes(B, Hq, Hkv, D, Lmax, num_splits)

@@ -10,12 +10,15 @@
 #include <cmath>
 #include <cstdint>
 #include <cstdlib>
+#include <map>
 #include <mutex>
+#include <tuple>
 
 #include "parallax.h"
 #include "parallax_testing.h"
 
 #include "common.cuh"
+#include "kernel_cluster.cuh"
 #include "kernel_copy.cuh"
 #include "kernel_generic.cuh"
 #include "kernel_merge.cuh"
@@ -295,6 +298,168 @@ int launch_merge(const Call& c, const DecodeParams& prm, int P) {
              : PARALLAX_ERR_CUDA;
 }
 
+// ------------------------------------------------------- cluster path --
+
+bool tma_path(const Call& c);
+
+// Dynamic shared memory of the cluster kernel for a group of G query heads.
+template <int D, bool PROBE>
+int cluster_smem_bytes(int G) {
+  const TcSmemLayout L =
+      tc_smem_layout(D, TcGeom<D>::kStageBytes, TcGeom<D>::kStages, G, PROBE);
+  return cluster_smem_total(L, G, D);
+}
+
+// Raises the kernel's shared-memory limit and allows clusters above the
+// portable size of 8, once per device.
+template <typename Kernel>
+int prepare_cluster_kernel(Kernel kernel, int smem, std::atomic<int>* done_dev) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PARALLAX_ERR_CUDA;
+  if (dev >= 0 && dev < 256 && done_dev[dev].load(std::memory_order_acquire) >= smem)
+    return PARALLAX_OK;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+          cudaSuccess ||
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+          cudaSuccess)
+    return PARALLAX_ERR_CUDA;
+  if (dev >= 0 && dev < 256) done_dev[dev].store(smem, std::memory_order_release);
+  return PARALLAX_OK;
+}
+
+template <int D, bool PROBE, bool OUT_F32>
+auto cluster_kernel() {
+  return parallax_cluster_kernel<D, PROBE, OUT_F32, PROBE || OUT_F32>;
+}
+
+template <int D, bool PROBE, bool OUT_F32>
+std::atomic<int>* cluster_prepared() {
+  static std::atomic<int> done[256];
+  return done;
+}
+
+// How many clusters of S CTAs of this kernel the current device holds at once
+// (cudaOccupancyMaxActiveClusters), cached per device, kernel, G and S.
+template <int D, bool PROBE, bool OUT_F32>
+int max_active_clusters(int G, int S, int* out) {
+  static std::mutex mu;
+  static std::map<std::tuple<int, int, int>, int> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PARALLAX_ERR_CUDA;
+  const auto key = std::make_tuple(dev, G, S);
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) {
+      *out = it->second;
+      return PARALLAX_OK;
+    }
+  }
+  auto kernel = cluster_kernel<D, PROBE, OUT_F32>();
+  const int smem = cluster_smem_bytes<D, PROBE>(G);
+  int st = prepare_cluster_kernel(kernel, smem, cluster_prepared<D, PROBE, OUT_F32>());
+  if (st != PARALLAX_OK) return st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)S;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)S);
+  cfg.blockDim = dim3(kTcThreads);
+  cfg.dynamicSmemBytes = (size_t)smem;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    n = 0;  // a size the device can not run: never chosen
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  cache[key] = n;
+  *out = n;
+  return PARALLAX_OK;
+}
+
+template <int D, bool PROBE, bool OUT_F32>
+int choose_cluster_impl(int items, int G, int sm, int* S_out) {
+  *S_out = 0;
+  if (items < 1 || items > sm / 2) return PARALLAX_OK;
+  for (int S = std::min(kClusterMax, sm / items); S >= 2; --S) {
+    int n = 0;
+    const int st = max_active_clusters<D, PROBE, OUT_F32>(G, S, &n);
+    if (st != PARALLAX_OK) return st;
+    if (n >= items) {
+      *S_out = S;
+      return PARALLAX_OK;
+    }
+  }
+  return PARALLAX_OK;
+}
+
+// The cluster size a call runs with (0: the split-KV + merge path). The
+// cluster path takes contiguous bf16 caches without a window, with the
+// default split (num_splits = 0), when every (batch row, kv head) item can
+// have a cluster of at least two CTAs resident at once.
+int cluster_plan(const Call& c, int* S) {
+  *S = 0;
+  if (c.kv_mode != kKvContiguous || c.window != 0 || c.phases != 3 || c.num_splits != 0 ||
+      env_splits() > 0 || !tma_path(c))
+    return PARALLAX_OK;
+  int sm = 0;
+  int st = current_sm_count(&sm);
+  if (st != PARALLAX_OK) return st;
+  const long long items = (long long)c.B * c.Hkv;
+  if (items > sm / 2) return PARALLAX_OK;
+  const int G = c.Hq / c.Hkv, it = (int)items;
+  const bool f32 = c.out_dtype == PARALLAX_DTYPE_F32;
+  if (c.D == 128) {
+    if (c.probe) return f32 ? choose_cluster_impl<128, true, true>(it, G, sm, S)
+                            : choose_cluster_impl<128, true, false>(it, G, sm, S);
+    return f32 ? choose_cluster_impl<128, false, true>(it, G, sm, S)
+               : choose_cluster_impl<128, false, false>(it, G, sm, S);
+  }
+  if (c.probe) return f32 ? choose_cluster_impl<64, true, true>(it, G, sm, S)
+                          : choose_cluster_impl<64, true, false>(it, G, sm, S);
+  return f32 ? choose_cluster_impl<64, false, true>(it, G, sm, S)
+             : choose_cluster_impl<64, false, false>(it, G, sm, S);
+}
+
+template <int D, bool PROBE, bool OUT_F32>
+int launch_cluster(const Call& c, const DecodeParams& prm, int S) {
+  auto kernel = cluster_kernel<D, PROBE, OUT_F32>();
+  const int smem = cluster_smem_bytes<D, PROBE>(prm.G);
+  int st = prepare_cluster_kernel(kernel, smem, cluster_prepared<D, PROBE, OUT_F32>());
+  if (st != PARALLAX_OK) return st;
+  CUtensorMap tmK, tmV;
+  if ((st = encode_cache_map(&tmK, c.k, D, c.Lmax, c.Hkv, c.B, c.kv_layout)) != PARALLAX_OK)
+    return st;
+  if ((st = encode_cache_map(&tmV, c.v, D, c.Lmax, c.Hkv, c.B, c.kv_layout)) != PARALLAX_OK)
+    return st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)S;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(c.B * c.Hkv * S));
+  cfg.blockDim = dim3(kTcThreads);
+  cfg.dynamicSmemBytes = (size_t)smem;
+  cfg.stream = c.stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, kernel, tmK, tmV, prm) == cudaSuccess ? PARALLAX_OK
+                                                                        : PARALLAX_ERR_CUDA;
+}
+
+template <bool PROBE, bool OUT_F32>
+int run_cluster(const Call& c, const DecodeParams& prm, int S) {
+  return c.D == 128 ? launch_cluster<128, PROBE, OUT_F32>(c, prm, S)
+                    : launch_cluster<64, PROBE, OUT_F32>(c, prm, S);
+}
+
 // The TMA kernel takes bf16 caches whose GQA group (q and r rows with the
 // probe) fits its 8 mma columns; everything else runs on the generic kernel.
 bool tma_path(const Call& c) {
@@ -328,12 +493,16 @@ int run_phases(const Call& c, const DecodeParams& prm, int P) {
 int run(const Call& c) {
   int st = validate(c);
   if (st != PARALLAX_OK) return st;
+  int S = 0;
+  if ((st = cluster_plan(c, &S)) != PARALLAX_OK) return st;
   int P = 0;
-  if ((st = resolve_splits(c.num_splits, c.B, c.Hkv, planned_len(c), !tma_path(c), &P)) !=
-      PARALLAX_OK)
+  if (S == 0 &&
+      (st = resolve_splits(c.num_splits, c.B, c.Hkv, planned_len(c), !tma_path(c), &P)) !=
+          PARALLAX_OK)
     return st;
   const int G = c.Hq / c.Hkv;
-  if (c.ws_bytes < workspace_bytes_for(G, c.D, P)) return PARALLAX_ERR_WORKSPACE_TOO_SMALL;
+  if (c.ws_bytes < (S > 0 ? kWorkspaceHeaderBytes : workspace_bytes_for(G, c.D, P)))
+    return PARALLAX_ERR_WORKSPACE_TOO_SMALL;
 
   DecodeParams prm{};
   prm.q = c.q;
@@ -370,6 +539,10 @@ int run(const Call& c) {
   prm.debug_skip_first_tile = c.debug_skip_first_tile;
 
   const bool f32 = c.out_dtype == PARALLAX_DTYPE_F32;
+  if (S > 0) {
+    if (c.probe) return f32 ? run_cluster<true, true>(c, prm, S) : run_cluster<true, false>(c, prm, S);
+    return f32 ? run_cluster<false, true>(c, prm, S) : run_cluster<false, false>(c, prm, S);
+  }
   if (c.probe) return f32 ? run_phases<true, true>(c, prm, P) : run_phases<true, false>(c, prm, P);
   return f32 ? run_phases<false, true>(c, prm, P) : run_phases<false, false>(c, prm, P);
 }
@@ -441,6 +614,31 @@ int parallax_default_splits(int B, int Hq, int Hkv, int Lmax, int in_dtype, int 
   c.probe = probe != 0;
   return choose_splits_impl(B, Hkv, Lmax, sm_count,
                             tma_path(c) ? kMinKeysPerSplit : kMinKeysPerSplitGeneric);
+}
+
+int parallax_decode_plan(int B, int Hq, int Hkv, int D, int Lmax, int in_dtype, int out_dtype,
+                         int probe, int* grid_ctas, int* cluster_ctas) {
+  if (!grid_ctas || !cluster_ctas) return PARALLAX_ERR_NULL_POINTER;
+  if (!shape_ok(B, Hq, Hkv, D, Lmax)) return PARALLAX_ERR_BAD_SHAPE;
+  if (D != 64 && D != 128) return PARALLAX_ERR_UNSUPPORTED_HEAD_DIM;
+  if ((in_dtype != PARALLAX_DTYPE_BF16 && in_dtype != PARALLAX_DTYPE_F32) ||
+      (out_dtype != PARALLAX_DTYPE_BF16 && out_dtype != PARALLAX_DTYPE_F32))
+    return PARALLAX_ERR_UNSUPPORTED_DTYPE;
+  Call c = make_call(3, probe != 0, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, B, Hq,
+                     Hkv, D, 1.f, nullptr, Lmax, in_dtype, out_dtype, 0, nullptr, 0);
+  int S = 0;
+  int st = cluster_plan(c, &S);
+  if (st != PARALLAX_OK) return st;
+  if (S > 0) {
+    *grid_ctas = B * Hkv * S;
+    *cluster_ctas = S;
+    return PARALLAX_OK;
+  }
+  int P = 0;
+  if ((st = resolve_splits(0, B, Hkv, Lmax, !tma_path(c), &P)) != PARALLAX_OK) return st;
+  *grid_ctas = P;
+  *cluster_ctas = 0;
+  return PARALLAX_OK;
 }
 
 size_t parallax_decode_workspace_bytes(int B, int Hq, int Hkv, int D, int Lmax, int num_splits) {

@@ -1,0 +1,136 @@
+"""GPU parity of the cluster schedule: for few (batch row, kv head) items a
+num_splits = 0 decode runs one thread-block cluster per item, the CTAs taking
+the item's 64-key tiles round-robin and combining their (m, l, b, A, C) in
+distributed shared memory, with no merge kernel. Checked against the fp64
+oracle (bf16 and fp32 outputs, Parallax and R = 0, GQA groups, both head
+sizes, lengths that end inside a tile, lengths shorter than one tile per CTA,
+empty and clamped lengths, NaN padding), against the split-KV + merge
+schedule, for determinism, and for its bounded waits."""
+import ctypes
+import time
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parameterized_local_linear_b200 import binding, inputs
+
+pytestmark = pytest.mark.gpu
+
+TOL = {torch.bfloat16: 2e-2, torch.float32: 1e-4}
+
+
+def scaled_error(got, ref):
+    g = got.detach().float().cpu().double().numpy()
+    assert np.all(np.isfinite(g)), "non-finite output"
+    return float(np.max(np.abs(g - ref) / np.maximum(1.0, np.abs(ref))))
+
+
+def plan(w, out_dtype=torch.bfloat16, probe=True):
+    return binding.parallax_decode_plan(w.B, w.Hq, w.Hkv, w.D, w.Lmax, w.dtype, out_dtype, probe)
+
+
+def test_plan_takes_clusters_for_one_sequence_and_partitions_for_a_large_batch():
+    q = plan(inputs.WORKLOADS["qwen"])
+    assert 2 <= q["cluster_ctas"] <= 16 and q["grid_ctas"] == 8 * q["cluster_ctas"]
+    big = plan(inputs.WORKLOADS["large"])
+    assert big["cluster_ctas"] == 0 and big["grid_ctas"] >= 1
+    fp32 = plan(inputs.WORKLOADS["tiny"])  # fp32 caches: the generic kernel's partitions
+    assert fp32["cluster_ctas"] == 0
+
+
+CASES = [
+    # B, Hq, Hkv, D, Lmax, lengths
+    (1, 16, 8, 128, 4096, (4096,)),        # the Qwen-3 decode step
+    (1, 16, 8, 128, 4000, (3999,)),        # ends inside a tile, Lmax not a tile multiple
+    (2, 32, 8, 128, 3000, (0, 2999)),      # an empty sequence, G = 4
+    (3, 8, 8, 64, 2048, (1, 65, 2048)),    # MHA, D = 64
+    (1, 4, 1, 128, 700, (700,)),           # G = 4, one item, fewer tiles than CTAs
+    (2, 16, 8, 64, 100, (37, 100)),        # a cache shorter than two tiles
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,D,Lmax,lengths", CASES)
+def test_cluster_matches_oracle(B, Hq, Hkv, D, Lmax, lengths):
+    w = inputs.custom_workload("cluster", B=B, Hq=Hq, Hkv=Hkv, D=D, Lmax=Lmax, lengths=lengths,
+                               seed=700 + B + Hq + D + Lmax, r_scale=1.0)
+    assert plan(w)["cluster_ctas"] >= 2, plan(w)
+    x = inputs.make_inputs(w, device="cuda")  # NaN padding past each length
+    ref = oracle.parallax_decode(x["q"], x["r"], x["k"], x["v"], x["seqlens"], x["scale"])
+    soft = oracle.softmax_decode(x["q"], x["k"], x["v"], x["seqlens"], x["scale"])
+    for out_dtype in (torch.bfloat16, torch.float32):
+        ws = binding.Workspace(B, Hq, Hkv, D, Lmax)
+        got = binding.parallax_decode(x["q"], x["r"], x["k"], x["v"], x["seqlens"],
+                                      scale=x["scale"], out_dtype=out_dtype, workspace=ws)
+        err = scaled_error(got, ref)
+        assert err <= TOL[out_dtype], (out_dtype, err)
+        for b, n in enumerate(lengths):
+            if n == 0:
+                assert torch.all(got[b] == 0)
+        got = binding.parallax_softmax_decode(x["q"], x["k"], x["v"], x["seqlens"],
+                                              scale=x["scale"], out_dtype=out_dtype, workspace=ws)
+        assert scaled_error(got, soft) <= TOL[out_dtype], out_dtype
+        assert ws.status() == (0, 0)
+
+
+def test_cluster_agrees_with_split_merge_and_is_deterministic():
+    w = inputs.WORKLOADS["qwen"]
+    x = inputs.make_inputs(w, device="cuda")
+    a = binding.parallax_decode(x["q"], x["r"], x["k"], x["v"], x["seqlens"], scale=x["scale"],
+                                out_dtype=torch.float32)
+    b = binding.parallax_decode(x["q"], x["r"], x["k"], x["v"], x["seqlens"], scale=x["scale"],
+                                out_dtype=torch.float32)
+    assert torch.equal(a, b)
+    P = binding.parallax_default_splits(w.B, w.Hq, w.Hkv, w.Lmax, w.dtype)
+    c = binding.parallax_decode(x["q"], x["r"], x["k"], x["v"], x["seqlens"], scale=x["scale"],
+                                out_dtype=torch.float32, num_splits=P)
+    d = (a.double() - c.double()).abs() / c.double().abs().clamp(min=1.0)
+    assert float(d.max()) <= 1e-4
+
+
+def test_cluster_clamps_and_reports_lengths():
+    w = inputs.custom_workload("cluster_clamp", B=2, Hq=16, Hkv=8, D=128, Lmax=300,
+                               lengths=(300, 120), seed=711)
+    x = inputs.make_inputs(w, device="cuda", pad_value=None)
+    assert plan(w)["cluster_ctas"] >= 2
+    ws = binding.Workspace(2, 16, 8, 128, 300)
+    bad = torch.tensor([10_000, -3], dtype=torch.int32, device="cuda")
+    got = binding.parallax_decode(x["q"], x["r"], x["k"], x["v"], bad, scale=x["scale"],
+                                  out_dtype=torch.float32, workspace=ws)
+    rc, bits = ws.status(clear=True)
+    assert bits & 2
+    clamped = torch.tensor([300, 0], dtype=torch.int32)
+    ref = oracle.parallax_decode(x["q"], x["r"], x["k"], x["v"], clamped, x["scale"])
+    assert scaled_error(got, ref) <= 1e-4
+    assert torch.all(got[1] == 0)
+
+
+def test_cluster_bounded_wait_gives_up_and_context_survives():
+    """The testing hook leaves the first stage of every CTA unfilled; the
+    consumers' wait runs out (50 ms), the timeout is recorded, both cluster
+    barriers are still reached, and a normal decode afterwards is correct."""
+    lib = binding.load_library()
+    fn = lib.parallax_testing_decode_stalled
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    fn.argtypes = [vp] * 6 + [i] * 4 + [ctypes.c_float, vp, i, i, vp, ctypes.c_size_t, i]
+    fn.restype = i
+    w = inputs.custom_workload("cluster_stall", B=2, Hq=16, Hkv=8, D=128, Lmax=512, seed=712)
+    assert plan(w)["cluster_ctas"] >= 2
+    x = inputs.make_inputs(w, device="cuda")
+    ws = binding.Workspace(2, 16, 8, 128, 512)
+    out = torch.empty((2, 16, 128), device="cuda", dtype=torch.bfloat16)
+    stream = torch.cuda.current_stream().cuda_stream
+    t0 = time.perf_counter()
+    rc = fn(x["q"].data_ptr(), x["r"].data_ptr(), x["k"].data_ptr(), x["v"].data_ptr(),
+            x["seqlens"].data_ptr(), out.data_ptr(), 2, 16, 8, 128, x["scale"], stream, 512, 0,
+            ws.ptr(), ws.nbytes, 50)
+    assert rc == 0
+    status, bits = ws.status(clear=True)
+    assert bits & 1 and status == -9
+    assert time.perf_counter() - t0 < 5.0
+    got = binding.parallax_decode(x["q"], x["r"], x["k"], x["v"], x["seqlens"], scale=x["scale"],
+                                  out_dtype=torch.float32, workspace=ws)
+    ref = oracle.parallax_decode(x["q"], x["r"], x["k"], x["v"], x["seqlens"], x["scale"])
+    assert scaled_error(got, ref) <= 1e-4
+    assert ws.status() == (0, 0)

@@ -134,14 +134,18 @@ def test_deterministic_and_phases():
     x = inputs.make_inputs(inputs.custom_workload("det", B=5, Hq=16, Hkv=8, D=128, Lmax=3000,
                                                   lengths="uniform", seed=7), device="cuda")
     ws = binding.Workspace(5, 16, 8, 128, 3000)
-    a = run(x, torch.bfloat16, ws=ws)
-    b = run(x, torch.bfloat16, ws=ws)
-    assert torch.equal(a, b), "two identical calls differ"
+    # the default schedule (40 items: one cluster each) and the split-KV +
+    # merge schedule at the default partition count are each deterministic
+    P = binding.parallax_default_splits(5, 16, 8, 3000)
+    for splits in (0, P):
+        a = run(x, torch.bfloat16, num_splits=splits, ws=ws)
+        b = run(x, torch.bfloat16, num_splits=splits, ws=ws)
+        assert torch.equal(a, b), f"two identical calls differ (num_splits={splits})"
     c = torch.empty_like(a)
     binding.parallax_decode_phase(1, True, x["q"], x["r"], x["k"], x["v"], x["seqlens"], c, ws,
-                                  scale=x["scale"])
+                                  scale=x["scale"], num_splits=P)
     binding.parallax_decode_phase(2, True, x["q"], x["r"], x["k"], x["v"], x["seqlens"], c, ws,
-                                  scale=x["scale"])
+                                  scale=x["scale"], num_splits=P)
     assert torch.equal(a, c), "phase 1 + phase 2 differs from one call"
     assert ws.status() == (0, 0)
 
