@@ -302,12 +302,11 @@ int launch_merge(const Call& c, const DecodeParams& prm, int P) {
 
 bool tma_path(const Call& c);
 
-// Dynamic shared memory of the cluster kernel for a group of G query heads.
-template <int D, bool PROBE>
-int cluster_smem_bytes(int G) {
-  const TcSmemLayout L =
-      tc_smem_layout(D, TcGeom<D>::kStageBytes, TcGeom<D>::kStages, G, PROBE);
-  return cluster_smem_total(L, G, D);
+// Dynamic shared memory of the cluster kernel for a group of G query heads
+// and clusters of S CTAs.
+template <int D>
+int cluster_smem_bytes(int G, int S) {
+  return cluster_layout(TcGeom<D>::kStageBytes, ClusterGeom<D>::kStages, G, D, S).total;
 }
 
 // Raises the kernel's shared-memory limit and allows clusters above the
@@ -356,7 +355,7 @@ int max_active_clusters(int G, int S, int* out) {
     }
   }
   auto kernel = cluster_kernel<D, PROBE, OUT_F32>();
-  const int smem = cluster_smem_bytes<D, PROBE>(G);
+  const int smem = cluster_smem_bytes<D>(G, S);
   int st = prepare_cluster_kernel(kernel, smem, cluster_prepared<D, PROBE, OUT_F32>());
   if (st != PARALLAX_OK) return st;
   cudaLaunchAttribute attr[1];
@@ -428,7 +427,7 @@ int cluster_plan(const Call& c, int* S) {
 template <int D, bool PROBE, bool OUT_F32>
 int launch_cluster(const Call& c, const DecodeParams& prm, int S) {
   auto kernel = cluster_kernel<D, PROBE, OUT_F32>();
-  const int smem = cluster_smem_bytes<D, PROBE>(prm.G);
+  const int smem = cluster_smem_bytes<D>(prm.G, S);
   int st = prepare_cluster_kernel(kernel, smem, cluster_prepared<D, PROBE, OUT_F32>());
   if (st != PARALLAX_OK) return st;
   CUtensorMap tmK, tmV;
