@@ -207,7 +207,7 @@ int parallax_decode_phase(int phase, int probe, const void* q, const void* r,
  *  - one thread-block cluster per (batch row, kv head) item, for few items
  *    (B * Hkv at most half the SM count) on the TMA kernel's inputs: the
  *    item's 64-key tiles are dealt round-robin to *cluster_ctas CTAs (2 to
- *    16, the most that leave every cluster resident at once), which combine
+ *    8, the most that leave every cluster resident at once), which combine
  *    their (m, l, b, A, C) through distributed shared memory; no merge
  *    kernel and no partial records; *grid_ctas = B * Hkv * *cluster_ctas.
  * The results of the two agree within the decode tolerances (the sums are

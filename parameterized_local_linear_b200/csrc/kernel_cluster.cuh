@@ -38,7 +38,11 @@
 
 namespace plx {
 
-constexpr int kClusterMax = 16;  // CTAs per cluster (above 8 needs the non-portable size)
+constexpr int kClusterMax = 16;  // CTAs per cluster the kernel takes (above 8: non-portable)
+// The largest size the host chooses by itself. Measured on a B200 at the
+// Qwen-3 B = 1 step (8 items, 64 tiles each): 8 CTAs per item (8 tiles each)
+// 6.62 us, 9 -> 6.87, 10 -> 6.75; 11 and more fit only 7 clusters at a time.
+constexpr int kClusterAuto = 8;
 
 template <int D>
 struct ClusterGeom {
@@ -226,33 +230,52 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncwarp();
   cluster_arrive_release();
   cluster_wait();
+  // W lanes per output value (W >= S, a power of two dividing 32), one
+  // source record each, reduced with shuffles; whole warps iterate together
   const float* const slot = reinterpret_cast<const float*>(gbase + L.off_slots);
-  for (int j = tid; j < L.per; j += kTcThreads) {
+  const int W = S <= 2 ? 2 : (S <= 4 ? 4 : (S <= 8 ? 8 : 16));
+  const int total = L.per * W;
+  for (int base0 = warp * 32; base0 < total; base0 += kTcThreads) {
+    const int idx = base0 + lane, j = idx / W, src = idx - j * W;
     const int gi = rank * L.per + j;
-    if (gi >= G * D) break;
-    const int h = gi / D, d = gi - h * D;
-    float M = kNegInf;
-    for (int s = 0; s < S; ++s) M = fmaxf(M, slot[s * L.slot_stride + 4 * h]);
-    float Lw = 0.f, Bw = 0.f, Aw = 0.f, Cw = 0.f;
-    for (int s = 0; s < S; ++s) {
-      const float4 hd = *reinterpret_cast<const float4*>(slot + s * L.slot_stride + 4 * h);
-      const float2 ac = *reinterpret_cast<const float2*>(slot + s * L.slot_stride + 4 * G + 2 * j);
-      const float w = hd.x == kNegInf ? 0.f : ex2_approx(hd.x - M);
-      Lw += w * hd.y;
-      Aw += w * ac.x;
+    const bool value = idx < total && gi < G * D;
+    const int h = value ? gi / D : 0, d = value ? gi - h * D : 0;
+    float m = kNegInf, l = 0.f, bb = 0.f, a = 0.f, c = 0.f;
+    if (value && src < S) {
+      const float4 hd = *reinterpret_cast<const float4*>(slot + src * L.slot_stride + 4 * h);
+      const float2 ac =
+          *reinterpret_cast<const float2*>(slot + src * L.slot_stride + 4 * G + 2 * j);
+      m = hd.x;
+      l = hd.y;
+      bb = hd.z;
+      a = ac.x;
+      c = ac.y;
+    }
+    float M = m;
+    for (int o = 1; o < W; o <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    const float w = m == kNegInf ? 0.f : ex2_approx(m - M);
+    l *= w;
+    a *= w;
+    bb *= w;
+    c *= w;
+    for (int o = 1; o < W; o <<= 1) {
+      l += __shfl_xor_sync(0xffffffffu, l, o);
+      a += __shfl_xor_sync(0xffffffffu, a, o);
       if (PROBE) {
-        Bw += w * hd.z;
-        Cw += w * ac.y;
+        bb += __shfl_xor_sync(0xffffffffu, bb, o);
+        c += __shfl_xor_sync(0xffffffffu, c, o);
       }
     }
-    const float inv = Lw > 0.f ? 1.f / Lw : 0.f;  // no attended key: o = 0
-    const float vbar = Aw * inv;
-    const float o = PROBE ? vbar + Cw * inv - (Bw * inv) * vbar : vbar;
-    const size_t oi = ((size_t)b * p.Hq + (size_t)g * G + h) * D + d;
-    if (OUT_F32)
-      static_cast<float*>(p.out)[oi] = o;
-    else
-      static_cast<__nv_bfloat16*>(p.out)[oi] = __float2bfloat16_rn(o);
+    if (value && src == 0) {
+      const float inv = l > 0.f ? 1.f / l : 0.f;  // no attended key: o = 0
+      const float vbar = a * inv;
+      const float o = PROBE ? vbar + c * inv - (bb * inv) * vbar : vbar;
+      const size_t oi = ((size_t)b * p.Hq + (size_t)g * G + h) * D + d;
+      if (OUT_F32)
+        static_cast<float*>(p.out)[oi] = o;
+      else
+        static_cast<__nv_bfloat16*>(p.out)[oi] = __float2bfloat16_rn(o);
+    }
   }
 }
 

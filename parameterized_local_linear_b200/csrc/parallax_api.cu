@@ -95,6 +95,18 @@ int env_splits() {
   return value;
 }
 
+// PARALLAX_CLUSTER (read once per process), for experiments: a value in
+// 2..16 forces that cluster size on the cluster path, -1 turns the cluster
+// path off; 0 when unset or invalid (the occupancy-based choice).
+int env_cluster() {
+  static const int value = [] {
+    const char* e = std::getenv("PARALLAX_CLUSTER");
+    const long v = e ? std::strtol(e, nullptr, 10) : 0;
+    return (v == -1 || (v >= 2 && v <= 16)) ? (int)v : 0;
+  }();
+  return value;
+}
+
 int choose_splits_impl(int B, int Hkv, int Lmax, int sm_count,
                        long long keys_per_split = kMinKeysPerSplit) {
   if (env_splits() > 0) return env_splits();
@@ -384,7 +396,7 @@ template <int D, bool PROBE, bool OUT_F32>
 int choose_cluster_impl(int items, int G, int sm, int* S_out) {
   *S_out = 0;
   if (items < 1 || items > sm / 2) return PARALLAX_OK;
-  for (int S = std::min(kClusterMax, sm / items); S >= 2; --S) {
+  for (int S = std::min(kClusterAuto, sm / items); S >= 2; --S) {
     int n = 0;
     const int st = max_active_clusters<D, PROBE, OUT_F32>(G, S, &n);
     if (st != PARALLAX_OK) return st;
@@ -403,13 +415,17 @@ int choose_cluster_impl(int items, int G, int sm, int* S_out) {
 int cluster_plan(const Call& c, int* S) {
   *S = 0;
   if (c.kv_mode != kKvContiguous || c.window != 0 || c.phases != 3 || c.num_splits != 0 ||
-      env_splits() > 0 || !tma_path(c))
+      env_splits() > 0 || env_cluster() < 0 || !tma_path(c))
     return PARALLAX_OK;
   int sm = 0;
   int st = current_sm_count(&sm);
   if (st != PARALLAX_OK) return st;
   const long long items = (long long)c.B * c.Hkv;
   if (items > sm / 2) return PARALLAX_OK;
+  if (env_cluster() > 0) {
+    *S = env_cluster();
+    return PARALLAX_OK;
+  }
   const int G = c.Hq / c.Hkv, it = (int)items;
   const bool f32 = c.out_dtype == PARALLAX_DTYPE_F32;
   if (c.D == 128) {
