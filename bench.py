@@ -879,15 +879,16 @@ class DecodeRig:
         self.use_graphs = self.nbuf > 1
         self.runners = {True: self._make_runner(True), False: self._make_runner(False)}
 
-    def step(self, b, probe=True):
+    def step(self, b, probe=True, out=None):
         bd = self.binding
+        out = self.out if out is None else out
         if probe:
             bd.parallax_decode(b["q"], b["r"], b["k"], b["v"], b["seqlens"], scale=b["scale"],
-                               out=self.out, num_splits=self.num_splits, workspace=self.ws,
+                               out=out, num_splits=self.num_splits, workspace=self.ws,
                                stream=self.stream)
         else:
             bd.parallax_softmax_decode(b["q"], b["k"], b["v"], b["seqlens"], scale=b["scale"],
-                                       out=self.out, num_splits=self.num_splits,
+                                       out=out, num_splits=self.num_splits,
                                        workspace=self.ws, stream=self.stream)
 
     def _make_runner(self, probe):
@@ -1156,7 +1157,8 @@ def main():
 
     # ---- end to end through the public API with host buffers ----
     # A step's inputs (q, r and the lengths) sit in one pinned host block and
-    # go over in one copy, into one device block whose views the call takes.
+    # go over in one copy, into one device block whose views the call takes;
+    # the output comes back every step.
     def packed_views(tensors, device):
         offs, n = [], 0
         for t in tensors:
@@ -1171,35 +1173,28 @@ def main():
     for hv, t in zip(host_views, (x["q"], x["r"], x["seqlens"])):
         hv.copy_(t.cpu())
     host_block = host_block.pin_memory()
-    dev_sets = []
-    for b in bufs:
-        dev_blk, (dq, dr, dsl) = packed_views([x["q"], x["r"], x["seqlens"]], dev)
-        dev_sets.append((dev_blk, {**b, "q": dq, "r": dr, "seqlens": dsl}))
-    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = host_block.numel()
     k_e2e = min(args.steps, 2000 if use_graphs else args.steps)
 
-    # Small per-step transfers go through parallax_copy (a kernel over the
-    # mapped pinned blocks: ~3 us each on the GPU timeline against ~8 us for a
-    # DMA copy of a few KB); large ones through DMA copies.
-    small = host_block.numel() + out_host.numel() * out_host.element_size() <= (1 << 20)
-    transfer = ("parallax_copy (kernel over mapped pinned host memory)" if small
-                else "cudaMemcpyAsync (DMA)")
-
-    def e2e_step(i):
-        dev_blk, b = dev_sets[i % nbuf]
-        if small:
-            binding.parallax_copy(dev_blk, host_block, stream=stream)
-        else:
-            dev_blk.copy_(host_block, non_blocking=True)
-        step(b)
-        if small:
-            binding.parallax_copy(out_host, out, stream=stream)
-        else:
-            out_host.copy_(out, non_blocking=True)
-
     if use_graphs:
-        # the same copies and launches, replayed from a CUDA graph as the
-        # device-resident steps are (a decode loop captures its copies too)
+        # Small per-step transfers (graph-replayed workloads) go through
+        # parallax_copy (a kernel over the mapped pinned blocks: ~3 us each on
+        # the GPU timeline against ~8 us for a DMA copy of a few KB), one step
+        # after another, replayed from a CUDA graph as the device-resident
+        # steps are (a decode loop captures its copies too).
+        out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        transfer = "parallax_copy (kernel over mapped pinned host memory), serial per step"
+        dev_sets = []
+        for b in bufs:
+            dev_blk, (dq, dr, dsl) = packed_views([x["q"], x["r"], x["seqlens"]], dev)
+            dev_sets.append((dev_blk, {**b, "q": dq, "r": dr, "seqlens": dsl}))
+
+        def e2e_step(i):
+            dev_blk, b = dev_sets[i % nbuf]
+            binding.parallax_copy(dev_blk, host_block, stream=stream)
+            step(b)
+            binding.parallax_copy(out_host, out, stream=stream)
+
         for i in range(nbuf):
             e2e_step(i)
         torch.cuda.synchronize()
@@ -1209,13 +1204,48 @@ def main():
                 e2e_step(i)
         k_e2e = max(nbuf, k_e2e // nbuf * nbuf)
 
-        def run_e2e(k):
+        def run_e2e(k, start_event=None):
             for _ in range(k // nbuf):
                 g_e2e.replay()
     else:
-        def run_e2e(k):
+        # Large transfers: DMA copies on two copy streams, double-buffered:
+        # step i's input copy overlaps step i-1's decode and its output copy
+        # step i+1's (the steps are independent batches, as in a serving loop
+        # that uploads the next batch while the current one runs).
+        transfer = ("cudaMemcpyAsync (DMA) on two copy streams, double-buffered: each step's "
+                    "input copy overlaps the previous step's decode, its output copy the next one's")
+        s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+        slots = []
+        for _ in range(2):
+            dev_blk, (dq, dr, dsl) = packed_views([x["q"], x["r"], x["seqlens"]], dev)
+            slots.append({"blk": dev_blk, "b": {**bufs[0], "q": dq, "r": dr, "seqlens": dsl},
+                          "out": torch.empty_like(out),
+                          "out_host": torch.empty(out.shape, dtype=out.dtype).pin_memory(),
+                          "in_ready": torch.cuda.Event(), "decoded": torch.cuda.Event(),
+                          "out_done": torch.cuda.Event()})
+        out_host = slots[0]["out_host"]
+
+        def run_e2e(k, start_event=None):
+            if start_event is not None:
+                s_in.wait_event(start_event)
             for i in range(k):
-                e2e_step(i)
+                sl = slots[i % 2]
+                if i >= 2:
+                    s_in.wait_event(sl["decoded"])  # decode i-2 has read this input block
+                with torch.cuda.stream(s_in):
+                    sl["blk"].copy_(host_block, non_blocking=True)
+                sl["in_ready"].record(s_in)
+                stream.wait_event(sl["in_ready"])
+                if i >= 2:
+                    stream.wait_event(sl["out_done"])  # output i-2 has left this block
+                step(sl["b"], out=sl["out"])
+                sl["decoded"].record(stream)
+                s_out.wait_event(sl["decoded"])
+                with torch.cuda.stream(s_out):
+                    sl["out_host"].copy_(sl["out"], non_blocking=True)
+                sl["out_done"].record(s_out)
+            for sl in slots[:min(k, 2)]:
+                stream.wait_event(sl["out_done"])  # the region ends with the last output home
 
     # the end-to-end loop is timed as a user runs it: launches and copies
     # enqueued as the host goes, no gate in front
@@ -1224,13 +1254,13 @@ def main():
     dist.barrier()
     ee0, ee1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ee0.record(stream)
-    run_e2e(k_e2e)
+    run_e2e(k_e2e, ee0)
     ee1.record(stream)
     ee1.synchronize()
+    torch.cuda.synchronize()
     dist.barrier()
     t_e2e = dist.max(ee0.elapsed_time(ee1) / 1e3)
     step(bufs[0])  # leave the resident buffers' result behind
-    h2d = host_block.numel()
     d2h = out_host.numel() * out_host.element_size()
 
     # ---- latency distribution, the pages' method: q50 (q05, q95) over trials ----
@@ -1270,7 +1300,6 @@ def main():
     # ---- the latency-bound Qwen step beside the default workload ----
     companion = None
     if args.workload != "qwen" and not args.no_companion:
-        del dev_sets, host_block, out_host
         companion = qwen_companion(dev, stream, dist)
 
     hbm_peak, peak_src = measured_peaks()

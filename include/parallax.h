@@ -137,8 +137,9 @@ size_t parallax_decode_workspace_bytes(int B, int Hq, int Hkv, int D, int Lmax,
 /*
  * The Parallax decode forward: out = vbar + C/l - (b/l) vbar per query head
  * (see the top of this file). r holds the probe rows, one per query head,
- * shaped like q. Launches the split-KV kernel and the split-merge kernel on
- * `stream`.
+ * shaped like q. Launches, on `stream`, either one cluster kernel (few
+ * (batch row, kv head) items) or the split-KV kernel and the split-merge
+ * kernel; parallax_decode_plan says which.
  */
 int parallax_decode(const void* q, const void* r, const void* k_cache,
                     const void* v_cache, const int32_t* cache_seqlens, void* out,
