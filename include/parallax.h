@@ -201,7 +201,8 @@ int parallax_decode_phase(int phase, int probe, const void* q, const void* r,
 
 /*
  * How a decode call with num_splits = 0 runs these shapes on the current
- * device (contiguous cache, no window). Two schedules exist:
+ * device (any key space: contiguous, windowed, paged or block-sparse rows).
+ * Two schedules exist:
  *  - split-KV + merge: *grid_ctas partitions of the flattened key range (one
  *    CTA each), partial records in the workspace, then the merge kernel;
  *    *cluster_ctas = 0.

@@ -6,10 +6,14 @@
 // from the lengths, writing partial records to global memory and a second
 // kernel that merges them. Here the S CTAs that share item (b, g) form one
 // cluster. CTA `rank` takes the item's 64-key tiles rank, rank + S,
-// rank + 2S, ... so its first tiles are known before the length is read: one
-// producer lane per stage issues the tiles that fit in the ring (and lie
-// inside the cache) right after the dependency wait, and the length is read
-// while they fly. The consumer warps are those of the split-KV kernel
+// rank + 2S, ... of the row's key space (partition.cuh: the cache row, its
+// last W keys with a sliding window, a paged row, or a block-sparse list;
+// paged and block-sparse tiles are resolved by tile_source and publish their
+// attended prefix per stage). On a contiguous row without a window the
+// first tiles are known before the length is read: one producer lane per
+// stage issues the tiles that fit in the ring (and lie inside the cache)
+// right after the dependency wait, and the length is read while they fly.
+// The consumer warps are those of the split-KV kernel
 // (TcConsumer: GQA-packed mma.sync scores and value products, online
 // (m, l, b, A, C)).
 //
@@ -66,8 +70,9 @@ __host__ __device__ inline ClusterLayout cluster_layout(int stage_bytes, int sta
   L.off_p = stages * stage_bytes;
   L.off_bar = L.off_p + kTcConsumers * 512;
   L.off_misc = align_up(L.off_bar + 8 * (2 * stages + 1), 16);  // full, empty, fin
-  L.off_slots = L.off_misc + 16;
+  L.off_slots = L.off_misc + 16 + 4 * stages;  // abort flag, then each stage's attended keys
   L.per = (G * D + S - 1) / S;
+  L.off_slots = align_up(L.off_slots, 16);
   L.slot_stride = align_up(4 * G + 2 * L.per, 4);  // floats; rows stay 16-byte aligned
   L.total = L.off_slots + S * L.slot_stride * 4 + 1024;  // + alignment slack
   return L;
@@ -99,6 +104,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t bar_empty = bar_full + 8 * kStages;
   const uint32_t bar_fin = bar_empty + 8 * kStages;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L.off_misc);
+  // paged / block-sparse rows: attended keys (a prefix) of the tile in each stage
+  volatile int* stage_valid = reinterpret_cast<volatile int*>(gbase + L.off_misc + 16);
   float* const merge_scr = reinterpret_cast<float*>(gbase);  // the drained ring
   const uint32_t slots = base + L.off_slots;
 
@@ -125,32 +132,47 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // what the previous kernel in the stream writes before this wait.
   pdl_wait_primary();
 
-  // tile j of this CTA is the item's tile rank + S j; the first ones that fit
-  // in the ring and lie inside the cache are issued before the length is known
+  // tile j of this CTA is the item's tile rank + S j; on a contiguous row
+  // without a window the first ones that fit in the ring and lie inside the
+  // cache are issued before the length is known
+  const KeySpace ks = key_space(p);
+  const bool contiguous = p.kv_mode == kKvContiguous;
   const int cache_tiles = (p.Lmax + kTileKeys - 1) / kTileKeys;
-  const int nspec = rank < cache_tiles ? min(kStages, (cache_tiles - rank + S - 1) / S) : 0;
+  const int nspec = (contiguous && p.window == 0 && rank < cache_tiles)
+                        ? min(kStages, (cache_tiles - rank + S - 1) / S)
+                        : 0;
   const bool skip0 = p.debug_skip_first_tile != 0;  // testing hook: stage 0 never filled
   bool ok = true;
 
   if (warp == kTcConsumers) {
     // ---------------------------------------------------------- producer --
-    auto issue = [&](int j) {
+    // tile j's first key and row on the K/V view: kbase + its position on a
+    // contiguous row, else where tile_source finds it (and its attended keys,
+    // published in the stage's word before the arrive below)
+    auto issue = [&](int j, int kbase) {
       const int stage = j % kStages;
       const uint32_t full = bar_full + 8 * stage;
       const uint32_t sK = base + stage * kStageBytes;
-      const int key = (rank + S * j) * kTileKeys;
+      int key = kbase + (rank + S * j) * kTileKeys, row = b;
+      if (!contiguous) {
+        int nv;
+        tile_source(p, b, (rank + S * j) * kTileKeys, &key, &row, &nv);
+        stage_valid[stage] = nv;
+      }
       mbar_arrive_expect_tx(full, kStageBytes);
-      tma_load_5d(sK, &tmK, 0, key, 0, g, b, full, policy);
-      tma_load_5d(sK + kKBytes, &tmV, 0, key, 0, g, b, full, policy);
+      tma_load_5d(sK, &tmK, 0, key, 0, g, row, full, policy);
+      tma_load_5d(sK + kKBytes, &tmV, 0, key, 0, g, row, full, policy);
     };
-    if (lane < nspec && !(lane == 0 && skip0)) issue(lane);  // fresh stages, one lane each
+    if (lane < nspec && !(lane == 0 && skip0)) issue(lane, 0);  // fresh stages, one lane each
     pdl_launch_dependents();
     __syncwarp();
     if (lane == 0) {
       uint32_t issued_mask = ((1u << nspec) - 1u) & (skip0 ? ~1u : ~0u), issued_par = 0;
-      const int n = p.seqlens ? clamp_len(__ldg(p.seqlens + b), p.Lmax) : p.Lmax;
-      const int ntiles = (n + kTileKeys - 1) / kTileKeys;
+      int kbase;
+      const int nkeys = item_keys(ks, b, &kbase);  // positions of the row's key space
+      const int ntiles = (nkeys + kTileKeys - 1) / kTileKeys;
       const int nreal = rank < ntiles ? (ntiles - rank + S - 1) / S : 0;
+      bool skip = skip0 && nspec == 0;
       for (int j = nspec; j < nreal; ++j) {
         const int stage = j % kStages;
         const uint32_t par = (uint32_t)(j / kStages) & 1u;
@@ -158,7 +180,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           ok = false;
           break;
         }
-        issue(j);
+        if (skip) {  // testing hook: the first stage is never filled
+          skip = false;
+          continue;
+        }
+        issue(j, kbase);
         issued_mask |= 1u << stage;
         issued_par = (issued_par & ~(1u << stage)) | (par << stage);
       }
@@ -177,11 +203,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   } else {
     // --------------------------------------------------------- consumers --
     pdl_launch_dependents();
-    const int nraw = p.seqlens ? __ldg(p.seqlens + b) : p.Lmax;
-    const int n = clamp_len(nraw, p.Lmax);
-    if (rank == 0 && tid == 0 && g == 0 && nraw != n)
+    if (rank == 0 && tid == 0 && g == 0 && item_clamped(ks, b))
       atomicOr(p.status, 2u /* PARALLAX_DEVICE_STATUS_SEQLEN_CLAMPED */);
-    const int ntiles = (n + kTileKeys - 1) / kTileKeys;
+    int kbase;
+    const int nkeys = item_keys(ks, b, &kbase);
+    const int ntiles = (nkeys + kTileKeys - 1) / kTileKeys;
     const int nreal = rank < ntiles ? (ntiles - rank + S - 1) / S : 0;
     const int J = max(nspec, nreal);
     const int group = warp / kConsumerWarps;
@@ -196,9 +222,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         ok = false;
         break;
       }
-      const int k0 = (rank + S * j) * kTileKeys;
+      const int k0 = (rank + S * j) * kTileKeys;  // position in the row's key space
       const uint32_t sK = base + stage * kStageBytes;
-      cs.tile(sK, sK + kKBytes, max(0, min(kTileKeys, n - k0)), p.scale_log2);
+      const int nvalid = contiguous ? max(0, min(kTileKeys, nkeys - k0)) : stage_valid[stage];
+      cs.tile(sK, sK + kKBytes, nvalid, p.scale_log2);
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_empty + 8 * stage);
     }

@@ -409,13 +409,14 @@ int choose_cluster_impl(int items, int G, int sm, int* S_out) {
 }
 
 // The cluster size a call runs with (0: the split-KV + merge path). The
-// cluster path takes contiguous bf16 caches without a window, with the
+// cluster path takes the TMA kernel's inputs (bf16 caches of any key space:
+// contiguous rows with or without a window, paged, block-sparse) with the
 // default split (num_splits = 0), when every (batch row, kv head) item can
 // have a cluster of at least two CTAs resident at once.
 int cluster_plan(const Call& c, int* S) {
   *S = 0;
-  if (c.kv_mode != kKvContiguous || c.window != 0 || c.phases != 3 || c.num_splits != 0 ||
-      env_splits() > 0 || env_cluster() < 0 || !tma_path(c))
+  if (c.phases != 3 || c.num_splits != 0 || env_splits() > 0 || env_cluster() < 0 ||
+      !tma_path(c))
     return PARALLAX_OK;
   int sm = 0;
   int st = current_sm_count(&sm);
@@ -447,10 +448,12 @@ int launch_cluster(const Call& c, const DecodeParams& prm, int S) {
   int st = prepare_cluster_kernel(kernel, smem, cluster_prepared<D, PROBE, OUT_F32>());
   if (st != PARALLAX_OK) return st;
   CUtensorMap tmK, tmV;
-  if ((st = encode_cache_map(&tmK, c.k, D, c.Lmax, c.Hkv, c.B, c.kv_layout)) != PARALLAX_OK)
-    return st;
-  if ((st = encode_cache_map(&tmV, c.v, D, c.Lmax, c.Hkv, c.B, c.kv_layout)) != PARALLAX_OK)
-    return st;
+  // a paged pool is viewed as a (kv_len, H, D) cache of page_size keys per page
+  const bool paged = c.kv_mode == kKvPaged;
+  const int rows = paged ? c.num_pages : c.B, len = paged ? c.page_size : c.Lmax;
+  const int layout = paged ? PARALLAX_KV_BSHD : c.kv_layout;
+  if ((st = encode_cache_map(&tmK, c.k, D, len, c.Hkv, rows, layout)) != PARALLAX_OK) return st;
+  if ((st = encode_cache_map(&tmV, c.v, D, len, c.Hkv, rows, layout)) != PARALLAX_OK) return st;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = (unsigned)S;

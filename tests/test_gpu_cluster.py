@@ -4,8 +4,10 @@ the item's 64-key tiles round-robin and combining their (m, l, b, A, C) in
 distributed shared memory, with no merge kernel. Checked against the fp64
 oracle (bf16 and fp32 outputs, Parallax and R = 0, GQA groups, both head
 sizes, lengths that end inside a tile, lengths shorter than one tile per CTA,
-empty and clamped lengths, NaN padding), against the split-KV + merge
-schedule, for determinism, and for its bounded waits."""
+empty and clamped lengths, NaN padding, and the other key spaces: a sliding
+window, a shuffled page pool, block-sparse lists with repeats and ids
+outside the cache), against the split-KV + merge schedule, for determinism,
+and for its bounded waits."""
 import ctypes
 import time
 
@@ -134,3 +136,86 @@ def test_cluster_bounded_wait_gives_up_and_context_survives():
     ref = oracle.parallax_decode(x["q"], x["r"], x["k"], x["v"], x["seqlens"], x["scale"])
     assert scaled_error(got, ref) <= 1e-4
     assert ws.status() == (0, 0)
+
+
+# --------------------------------------- other key spaces on the cluster path --
+
+def _windowed(x, W):
+    """The cache holding only each row's last min(n, W) keys, for the oracle."""
+    n = x["seqlens"].cpu().to(torch.int64)
+    k, v = torch.zeros_like(x["k"]), torch.zeros_like(x["v"])
+    for b in range(k.shape[0]):
+        e = int(n[b]); s = max(0, e - W)
+        k[b, :, :e - s] = x["k"][b, :, s:e]
+        v[b, :, :e - s] = x["v"][b, :, s:e]
+    return dict(x, k=k, v=v, seqlens=(n - (n - W).clamp(min=0)).to(torch.int32))
+
+
+@pytest.mark.parametrize("W", [1, 200, 5000])
+def test_cluster_sliding_window(W):
+    w = inputs.custom_workload("cluster_win", B=2, Hq=16, Hkv=8, D=128, Lmax=3000,
+                               lengths=(3000, 777), seed=720 + W, r_scale=1.0)
+    x = inputs.make_inputs(w, device="cuda")
+    assert plan(w)["cluster_ctas"] >= 2
+    y = _windowed(x, W)
+    want = oracle.parallax_decode(y["q"], y["r"], y["k"], y["v"], y["seqlens"], y["scale"])
+    for out_dtype in (torch.bfloat16, torch.float32):
+        got = binding.parallax_decode(x["q"], x["r"], x["k"], x["v"], x["seqlens"],
+                                      scale=x["scale"], out_dtype=out_dtype, window=W)
+        assert scaled_error(got, want) <= TOL[out_dtype], (W, out_dtype)
+
+
+@pytest.mark.parametrize("page_size", [64, 256])
+def test_cluster_paged(page_size):
+    """One sequence's pages scattered through a pool (the Qwen-3 shape), and
+    three sequences of ragged lengths: the cluster path against the oracle,
+    and against the split-KV + merge path."""
+    for w in (inputs.custom_workload("cluster_paged1", B=1, Hq=16, Hkv=8, D=128, Lmax=4096,
+                                     seed=730, r_scale=1.0),
+              inputs.custom_workload("cluster_paged3", B=3, Hq=16, Hkv=8, D=128, Lmax=2048,
+                                     lengths=(1, 1000, 2048), seed=731, r_scale=1.0)):
+        assert plan(w)["cluster_ctas"] >= 2
+        x = inputs.make_paged(w, page_size, "cuda")
+        want = oracle.parallax_decode_paged(x["q"], x["r"], x["k"], x["v"], x["table"],
+                                            x["seqlens"], x["scale"])
+        for out_dtype in (torch.bfloat16, torch.float32):
+            ws = binding.Workspace(w.B, w.Hq, w.Hkv, w.D, x["table"].shape[1] * page_size)
+            got = binding.parallax_decode_paged(x["q"], x["r"], x["k"], x["v"], x["table"],
+                                                x["seqlens"], scale=x["scale"],
+                                                out_dtype=out_dtype, workspace=ws)
+            assert scaled_error(got, want) <= TOL[out_dtype], (w.name, page_size, out_dtype)
+            assert ws.status() == (0, 0)
+        split = binding.parallax_decode_paged(x["q"], x["r"], x["k"], x["v"], x["table"],
+                                              x["seqlens"], scale=x["scale"],
+                                              out_dtype=torch.float32, num_splits=23)
+        assert scaled_error(got, split.double().cpu().numpy()) <= 1e-4
+
+
+def test_cluster_block_sparse_and_bad_ids():
+    w = inputs.custom_workload("cluster_bs", B=2, Hq=16, Hkv=8, D=128, Lmax=4096,
+                               lengths=(4096, 1500), seed=740, r_scale=1.0)
+    assert plan(w)["cluster_ctas"] >= 2
+    x = inputs.make_inputs(w, device="cuda")
+    ids = torch.tensor([[5, 0, 63, 17, 17, 40], [1, 22, 30, 0, 0, 0]], dtype=torch.int32)
+    cnt = torch.tensor([6, 3], dtype=torch.int32)
+    want = oracle.parallax_decode_block_sparse(x["q"], x["r"], x["k"], x["v"], ids.numpy(),
+                                               cnt.numpy(), x["seqlens"], x["scale"])
+    ws = binding.Workspace(2, 16, 8, 128, 64 * 6)
+    for out_dtype in (torch.bfloat16, torch.float32):
+        got = binding.parallax_decode_block_sparse(x["q"], x["r"], x["k"], x["v"], ids.cuda(),
+                                                   cnt.cuda(), x["seqlens"], scale=x["scale"],
+                                                   out_dtype=out_dtype, workspace=ws)
+        assert scaled_error(got, want) <= TOL[out_dtype], out_dtype
+        assert ws.status() == (0, 0)
+    bad = ids.clone()
+    bad[1, 1] = 1000  # outside the cache: left out and reported
+    got = binding.parallax_decode_block_sparse(x["q"], x["r"], x["k"], x["v"], bad.cuda(),
+                                               cnt.cuda(), x["seqlens"], scale=x["scale"],
+                                               out_dtype=torch.float32, workspace=ws)
+    rc, bits = ws.status(clear=True)
+    assert bits & 2
+    want_bad = oracle.parallax_decode_block_sparse(
+        x["q"], x["r"], x["k"], x["v"], torch.tensor([[5, 0, 63, 17, 17, 40], [1, 30, 0, 0, 0, 0]],
+                                                     dtype=torch.int32).numpy(),
+        torch.tensor([6, 2], dtype=torch.int32).numpy(), x["seqlens"], x["scale"])
+    assert scaled_error(got, want_bad) <= 1e-4
