@@ -688,6 +688,7 @@ def run_kv_variant(args):
         host_block[o:o + n_].copy_(x[k].cpu().contiguous().view(-1).view(torch.uint8))
         x[k] = dev_block[o:o + n_].view(x[k].dtype).view(x[k].shape)
     host_block = host_block.pin_memory()
+    dev_block.copy_(host_block)  # the views that now stand for q, r and the lengths hold them
     out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     small = nb + out_host.numel() * out_host.element_size() <= (1 << 20)
     transfer = ("parallax_copy (kernel over mapped pinned host memory)" if small
