@@ -239,3 +239,18 @@ def test_merge_many_pieces_and_workspace_reuse():
                                             num_splits=splits, workspace=ws)
         assert_close(b, soft, 1e-4, f"softmax, {splits} splits")
     assert ws.status() == (0, 0)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("Hq,Hkv", [(16, 8), (16, 4)])
+def test_fp32_output_large_probe_few_keys(D, Hq, Hkv):
+    """The fp32-output bound where the weights' rounding weighs most: r at
+    twice the large configs' scale (|s| ~ 2 sqrt(D)) and rows of 1 to 300
+    keys, on the cluster schedule (num_splits = 0) and the split-KV + merge
+    schedule."""
+    w = inputs.custom_workload("few", B=6, Hq=Hq, Hkv=Hkv, D=D, Lmax=300,
+                               lengths=(1, 2, 5, 17, 64, 300), seed=900 + D + Hkv, r_scale=2.0)
+    x = inputs.make_inputs(w, device="cuda")
+    ref = ref_parallax(x)
+    for splits in (0, 7):
+        assert_close(run(x, torch.float32, splits), ref, 1e-4, f"D={D} G={Hq // Hkv} {splits}")
