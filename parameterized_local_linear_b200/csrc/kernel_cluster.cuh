@@ -22,13 +22,18 @@
 //     combine them into this CTA's (M, L, B, A_d, C_d) per query head;
 //  2. the G*D output values of the item are dealt to the S CTAs in slices;
 //     each CTA pushes its combined values of slice o into CTA o's shared
-//     memory (st.shared::cluster; the cluster barrier's first phase, arrived
-//     at the start and waited for here, guarantees every CTA is running);
-//  3. one cluster barrier (release / acquire); CTA o then finishes its slice
-//     from the S records in its own shared memory:
+//     memory with st.async, whose bytes count off CTA o's "slots" mbarrier as
+//     they land (the cluster barrier, arrived at the start and waited for
+//     here, guarantees every CTA is running with its barriers initialised);
+//  3. CTA o waits on its own mbarrier for the bytes of all S sources (armed
+//     with their total at the start; every source pushes on every path, also
+//     after a timed-out wait, so the count always completes), then finishes
+//     its slice from the S records in its own shared memory:
 //       M = max m_s, w_s = 2^(m_s - M), l = sum w_s l_s (likewise b, A, C),
-//       o = A/l + C/l - (b/l)(A/l)   (A/l without the probe; 0 when l = 0),
-//     and no shared memory of another CTA is touched after that barrier.
+//       o = A/l + C/l - (b/l)(A/l)   (A/l without the probe; 0 when l = 0).
+//     A release barrier after the pushes is not needed: a sender only leaves
+//     once its own incoming bytes have landed, and nothing reads a sender's
+//     shared memory.
 //
 // Tiles past the item's length that were issued before the length was known
 // are consumed with zero attended keys. Every mbarrier wait is bounded; every
@@ -69,7 +74,7 @@ __host__ __device__ inline ClusterLayout cluster_layout(int stage_bytes, int sta
   ClusterLayout L{};
   L.off_p = stages * stage_bytes;
   L.off_bar = L.off_p + kTcConsumers * 512;
-  L.off_misc = align_up(L.off_bar + 8 * (2 * stages + 1), 16);  // full, empty, fin
+  L.off_misc = align_up(L.off_bar + 8 * (2 * stages + 2), 16);  // full, empty, fin, slots
   L.off_slots = L.off_misc + 16 + 4 * stages;  // abort flag, then each stage's attended keys
   L.per = (G * D + S - 1) / S;
   L.off_slots = align_up(L.off_slots, 16);
@@ -103,6 +108,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t bar_full = base + L.off_bar;
   const uint32_t bar_empty = bar_full + 8 * kStages;
   const uint32_t bar_fin = bar_empty + 8 * kStages;
+  const uint32_t bar_slots = bar_fin + 8;  // the pushes into this CTA's slots
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L.off_misc);
   // paged / block-sparse rows: attended keys (a prefix) of the tile in each stage
   volatile int* stage_valid = reinterpret_cast<volatile int*>(gbase + L.off_misc + 16);
@@ -115,8 +121,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(bar_empty + 8 * s, kConsumerWarps);
     }
     mbar_init(bar_fin, kTcConsumers);
+    mbar_init(bar_slots, 1);
     *abort_flag = 0;
     mbar_fence_init();
+    // the bytes S sources push into this CTA's slice: G headers of 16 bytes
+    // and an (A, C) pair of 8 bytes per value of the slice
+    const int nvals = min(L.per, G * D - rank * L.per);
+    mbar_arrive_expect_tx(bar_slots, (uint32_t)(S * (16 * G + 8 * max(nvals, 0))));
   }
   uint64_t policy = 0;
   if (warp == kTcConsumers) {
@@ -127,7 +138,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     policy = l2_policy_evict_first();
   }
   __syncthreads();
-  cluster_arrive_relaxed();  // phase 0: this CTA runs; its shared memory may be written
+  cluster_arrive_release();  // phase 0: this CTA runs, its barriers initialised
   // Launched with programmatic stream serialisation: nothing below may read
   // what the previous kernel in the stream writes before this wait.
   pdl_wait_primary();
@@ -245,18 +256,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       float M, Lw, Bw, Aw, Cw;
       tc_combine_warps<D, PROBE>(merge_scr, G, h, d, M, Lw, Bw, Aw, Cw);
       const int o = idx / L.per, j = idx - o * L.per;
-      st_cluster_f32x2(cluster_map(slots + (row + 4 * G + 2 * j) * 4u, (uint32_t)o), Aw, Cw);
+      st_async_f32x2(cluster_map(slots + (row + 4 * G + 2 * j) * 4u, (uint32_t)o), Aw, Cw,
+                     cluster_map(bar_slots, (uint32_t)o));
       if (d == 0) {
         for (int t = 0; t < S; ++t)
-          st_cluster_f32x4(cluster_map(slots + (row + 4 * h) * 4u, (uint32_t)t), M, Lw, Bw, 0.f);
+          st_async_f32x4(cluster_map(slots + (row + 4 * h) * 4u, (uint32_t)t), M, Lw, Bw, 0.f,
+                         cluster_map(bar_slots, (uint32_t)t));
       }
     }
   }
 
-  // 3. the cluster's pushes are visible; finish this CTA's slice locally
-  __syncwarp();
-  cluster_arrive_release();
-  cluster_wait();
+  // 3. this CTA's slice has landed (bounded wait, no abort shortcut: every
+  // source pushes, and this CTA must not leave before its bytes arrive)
+  if (!mbar_wait_bounded(bar_slots, 0, p.timeout_ns, nullptr)) {
+    if (tid == 0) atomicOr(p.status, 1u /* PARALLAX_DEVICE_STATUS_TIMEOUT */);
+    return;
+  }
   // W lanes per output value (W >= S, a power of two dividing 32), one
   // source record each, reduced with shuffles; whole warps iterate together
   const float* const slot = reinterpret_cast<const float*>(gbase + L.off_slots);

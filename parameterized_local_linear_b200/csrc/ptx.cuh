@@ -222,6 +222,28 @@ __device__ __forceinline__ void st_cluster_f32x2(uint32_t addr, float a, float b
                : "memory");
 }
 
+// Asynchronous store into another CTA's shared memory (addresses from
+// cluster_map) that counts its bytes off that CTA's mbarrier `remote_bar`
+// when it lands (complete_tx): the receiver waits on its own barrier, and the
+// sender needs no release fence.
+__device__ __forceinline__ void st_async_f32x2(uint32_t remote_addr, float a, float b,
+                                               uint32_t remote_bar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];" ::"r"(
+          remote_addr),
+      "f"(a), "f"(b), "r"(remote_bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void st_async_f32x4(uint32_t remote_addr, float a, float b, float c,
+                                               float d, uint32_t remote_bar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, "
+      "[%5];" ::"r"(remote_addr),
+      "f"(a), "f"(b), "f"(c), "f"(d), "r"(remote_bar)
+      : "memory");
+}
+
 // The address of the same shared-memory location in CTA `rank` of the cluster.
 __device__ __forceinline__ uint32_t cluster_map(uint32_t addr, uint32_t rank) {
   uint32_t r;

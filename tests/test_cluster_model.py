@@ -14,8 +14,9 @@ rank, rank + S, ... of the row's key space. Checked here:
   fill j - stages;
 - the output values of the item (G heads x D dims) are dealt to the S CTAs in
   slices that cover each value exactly once; every push lands inside the
-  owner's slot area, header and value rows do not overlap, and the area fits
-  in the kernel's shared memory;
+  owner's slot area, header and value rows do not overlap, the bytes an
+  owner's barrier expects equal the bytes its sources push, and the area
+  fits in the kernel's shared memory;
 - the reduction lanes (W >= S per value) stay inside whole warps.
 """
 import itertools
@@ -40,7 +41,7 @@ def layout(D, G, S):
     stages = STAGES[D]
     off_p = stages * STAGE_BYTES[D]
     off_bar = off_p + CONSUMER_WARPS * 512
-    off_misc = align_up(off_bar + 8 * (2 * stages + 1), 16)
+    off_misc = align_up(off_bar + 8 * (2 * stages + 2), 16)
     off_slots = align_up(off_misc + 16 + 4 * stages, 16)
     per = (G * D + S - 1) // S
     stride = align_up(4 * G + 2 * per, 4)
@@ -107,6 +108,11 @@ def test_slices_slots_and_shared_memory(D, G):
         # every value owned exactly once: owner o holds its consecutive slice
         covered = sorted(o * L["per"] + j for o, js in owners.items() for j in js)
         assert covered == list(range(G * D))
+        # the bytes each owner arms its barrier with = the bytes its sources push
+        for o in range(S):
+            nvals = max(0, min(L["per"], G * D - o * L["per"]))
+            pushed = S * (16 * G + 8 * len(owners.get(o, ())))
+            assert pushed == S * (16 * G + 8 * nvals)
 
 
 def test_reduction_lanes_stay_in_whole_warps():
