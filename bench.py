@@ -674,8 +674,9 @@ def run_kv_variant(args):
     if rc != 0:
         raise SystemExit(f"device status after timing: {binding.parallax_status_string(rc)}")
     # end to end: q, r and lengths packed in one pinned host block copied in,
-    # the output copied back, every step (small blocks through parallax_copy,
-    # as in the contiguous bench); the step then reads the device views
+    # the output copied back, every step (small pools through parallax_copy,
+    # large ones by DMA, as in the contiguous bench); the step reads device
+    # views of the copied block
     names = ("q", "r", "seqlens")
     offs, nb = [], 0
     for k in names:
@@ -690,30 +691,61 @@ def run_kv_variant(args):
     host_block = host_block.pin_memory()
     dev_block.copy_(host_block)  # the views that now stand for q, r and the lengths hold them
     out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    small = nb + out_host.numel() * out_host.element_size() <= (1 << 20)
-    transfer = ("parallax_copy (kernel over mapped pinned host memory)" if small
-                else "cudaMemcpyAsync (DMA)")
-
-    def e2e_step(i):
-        if small:
-            binding.parallax_copy(dev_block, host_block, stream=stream)
-        else:
-            dev_block.copy_(host_block, non_blocking=True)
-        step(True, i)
-        if small:
-            binding.parallax_copy(out_host, out, stream=stream)
-        else:
-            out_host.copy_(out, non_blocking=True)
-
     k_e2e = min(args.steps, 50)
+
+    def decode_with(xx, kk, vv, dst):
+        if args.kv_mode == "paged":
+            binding.parallax_decode_paged(xx["q"], xx["r"], kk, vv, xx["table"], xx["seqlens"],
+                                          scale=xx["scale"], out=dst, workspace=ws,
+                                          num_splits=args.num_splits, stream=stream)
+        else:
+            binding.parallax_decode_block_sparse(xx["q"], xx["r"], kk, vv, xx["block_ids"],
+                                                 xx["num_blocks"], xx["seqlens"],
+                                                 scale=xx["scale"], out=dst, workspace=ws,
+                                                 num_splits=args.num_splits, stream=stream)
+
     if nbuf > 1:
-        for i in range(nbuf):
-            e2e_step(i)
+        # small pools: per step its own input block and output buffer, the
+        # input copy on a side stream ahead of the decode and the output copy
+        # on another behind it (parallax_copy), replayed from a CUDA graph, as
+        # in the contiguous bench
+        transfer = ("parallax_copy (kernel over mapped pinned host memory) on two side streams, "
+                    "each step's input and output copies overlapping its neighbours' decodes")
+        s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+        sets = []
+        for _ in range(nbuf):
+            blk = torch.zeros(nb, dtype=torch.uint8, device=dev)
+            views = {k: blk[o:o + x[k].numel() * x[k].element_size()].view(x[k].dtype)
+                     .view(x[k].shape) for k, o in zip(names, offs)}
+            sets.append((blk, {**x, **views}, torch.empty_like(out),
+                         torch.empty(out.shape, dtype=out.dtype).pin_memory()))
+        ev_in = [torch.cuda.Event() for _ in range(nbuf)]
+        ev_dec = [torch.cuda.Event() for _ in range(nbuf)]
+        ev_out = [torch.cuda.Event() for _ in range(nbuf)]
+
+        def chain():
+            fork = torch.cuda.Event()
+            fork.record(stream)
+            s_in.wait_event(fork)
+            s_out.wait_event(fork)
+            for i in range(nbuf):
+                blk, xx, dout, hout = sets[i]
+                binding.parallax_copy(blk, host_block, stream=s_in)
+                ev_in[i].record(s_in)
+                stream.wait_event(ev_in[i])
+                decode_with(xx, kvs[i][0], kvs[i][1], dout)
+                ev_dec[i].record(stream)
+                s_out.wait_event(ev_dec[i])
+                binding.parallax_copy(hout, dout, stream=s_out)
+                ev_out[i].record(s_out)
+            for i in range(nbuf):
+                stream.wait_event(ev_out[i])
+
+        chain()
         torch.cuda.synchronize()
         g_e2e = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g_e2e, stream=stream):
-            for i in range(nbuf):
-                e2e_step(i)
+            chain()
         k_e2e = max(nbuf, k_e2e // nbuf * nbuf)
 
         def run_e2e(k_steps, start_event=None):
@@ -736,19 +768,6 @@ def run_kv_variant(args):
                           "in_ready": torch.cuda.Event(), "decoded": torch.cuda.Event(),
                           "out_done": torch.cuda.Event()})
 
-        def decode_into(xx, dst):
-            if args.kv_mode == "paged":
-                binding.parallax_decode_paged(xx["q"], xx["r"], xx["k"], xx["v"], xx["table"],
-                                              xx["seqlens"], scale=xx["scale"], out=dst,
-                                              workspace=ws, num_splits=args.num_splits,
-                                              stream=stream)
-            else:
-                binding.parallax_decode_block_sparse(xx["q"], xx["r"], xx["k"], xx["v"],
-                                                     xx["block_ids"], xx["num_blocks"],
-                                                     xx["seqlens"], scale=xx["scale"], out=dst,
-                                                     workspace=ws, num_splits=args.num_splits,
-                                                     stream=stream)
-
         def run_e2e(k_steps, start_event=None):
             if start_event is not None:
                 s_in.wait_event(start_event)
@@ -762,7 +781,7 @@ def run_kv_variant(args):
                 stream.wait_event(sl["in_ready"])
                 if i >= 2:
                     stream.wait_event(sl["out_done"])
-                decode_into(sl["x"], sl["out"])
+                decode_with(sl["x"], x["k"], x["v"], sl["out"])
                 sl["decoded"].record(stream)
                 s_out.wait_event(sl["decoded"])
                 with torch.cuda.stream(s_out):
@@ -1238,29 +1257,49 @@ def main():
     if use_graphs:
         # Small per-step transfers (graph-replayed workloads) go through
         # parallax_copy (a kernel over the mapped pinned blocks: ~3 us each on
-        # the GPU timeline against ~8 us for a DMA copy of a few KB), one step
-        # after another, replayed from a CUDA graph as the device-resident
-        # steps are (a decode loop captures its copies too).
-        out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        transfer = "parallax_copy (kernel over mapped pinned host memory), serial per step"
+        # the GPU timeline against ~8 us for a DMA copy of a few KB). Each
+        # step of a chain has its own input block and output buffer; its input
+        # copy runs on a side stream ahead of its decode and its output copy on
+        # another behind it, so the copies of neighbouring steps overlap the
+        # decode (the steps are independent batches, as in a serving loop).
+        # The chain is replayed from a CUDA graph as the device-resident steps
+        # are; every step's two copies are inside the timed region.
+        transfer = ("parallax_copy (kernel over mapped pinned host memory) on two side streams, "
+                    "each step's input and output copies overlapping its neighbours' decodes")
+        s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
         dev_sets = []
         for b in bufs:
             dev_blk, (dq, dr, dsl) = packed_views([x["q"], x["r"], x["seqlens"]], dev)
-            dev_sets.append((dev_blk, {**b, "q": dq, "r": dr, "seqlens": dsl}))
+            dev_sets.append((dev_blk, {**b, "q": dq, "r": dr, "seqlens": dsl}, torch.empty_like(out),
+                             torch.empty(out.shape, dtype=out.dtype).pin_memory()))
+        out_host = dev_sets[0][3]
+        ev_in = [torch.cuda.Event() for _ in range(nbuf)]
+        ev_dec = [torch.cuda.Event() for _ in range(nbuf)]
+        ev_out = [torch.cuda.Event() for _ in range(nbuf)]
 
-        def e2e_step(i):
-            dev_blk, b = dev_sets[i % nbuf]
-            binding.parallax_copy(dev_blk, host_block, stream=stream)
-            step(b)
-            binding.parallax_copy(out_host, out, stream=stream)
+        def chain():
+            fork = torch.cuda.Event()
+            fork.record(stream)
+            s_in.wait_event(fork)
+            s_out.wait_event(fork)
+            for i in range(nbuf):
+                dev_blk, b, dout, hout = dev_sets[i]
+                binding.parallax_copy(dev_blk, host_block, stream=s_in)
+                ev_in[i].record(s_in)
+                stream.wait_event(ev_in[i])
+                step(b, out=dout)
+                ev_dec[i].record(stream)
+                s_out.wait_event(ev_dec[i])
+                binding.parallax_copy(hout, dout, stream=s_out)
+                ev_out[i].record(s_out)
+            for i in range(nbuf):  # the chain ends with every output home
+                stream.wait_event(ev_out[i])
 
-        for i in range(nbuf):
-            e2e_step(i)
+        chain()
         torch.cuda.synchronize()
         g_e2e = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g_e2e, stream=stream):
-            for i in range(nbuf):
-                e2e_step(i)
+            chain()
         k_e2e = max(nbuf, k_e2e // nbuf * nbuf)
 
         def run_e2e(k, start_event=None):
