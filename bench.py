@@ -136,6 +136,15 @@ def measured_bf16_peak():
         return FALLBACK_BF16_TFLOPS, "fallback"
 
 
+def measured_bf16_sustained():
+    """Dense bf16 tensor peak held for seconds under the power cap, or None."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops_sustained"])
+    except Exception:
+        return None
+
+
 # ncu summaries whose traffic line the bench reports, per (workload, kernel):
 # (file, batch rows the capture ran). A capture on fewer rows than the
 # workload is scaled by the rows processed (every row of these workloads has
@@ -436,7 +445,9 @@ def run_prefill(args):
                           device=dev)
     out = torch.empty_like(q)
     out_f32 = out.dtype == torch.float32
-    ws = torch.zeros(256, dtype=torch.uint8, device=dev)
+    # room for the fp16 copy of V (the fp16 value products of the bf16 output)
+    ws = (binding.prefill_workspace(B, L, Hkv, D, dev) if lens is None
+          else binding.prefill_workspace(1, sum(lens), Hkv, D, dev))
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     in_bytes = sum(t.numel() * t.element_size() for t in (q, r, k, v, out))
     # inputs smaller than the L2: rotate over enough copies to exceed twice the L2
@@ -543,6 +554,7 @@ def run_prefill(args):
         cpu = {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc}
 
     peak, peak_src = measured_bf16_peak()
+    sustained = measured_bf16_sustained()
     N = dist.world
     achieved = flops / kern_s / 1e12
     clocks = sampler.summary()
@@ -550,7 +562,9 @@ def run_prefill(args):
         "metric": PREFILL_METRIC, "value": N * flops * args.steps / t_step / 1e12,
         "unit": "TFLOP/s", "n_gpus": N, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": t_step / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        # bf16 scores; bf16 output: value products on fp16 weights and V (the
+        # exact bf16 hi + lo pair on tiles outside fp16's range)
+        "vs_baseline": None, "dtype": "bf16+f16", "data": "synthetic",
         "config": dict(cfg, parallelism=f"replicas x{N}" if N > 1 else "single GPU",
                        l2=(f"rotate {nbuf} input copies ({nbuf * in_bytes / 1e6:.0f} MB > 2x L2)"
                            if nbuf > 1 else f"inputs ({in_bytes / 1e6:.0f} MB) larger than L2")),
@@ -560,12 +574,16 @@ def run_prefill(args):
         "e2e": {"value": N * flops * k_e2e / t_e2e / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "us_per_step": t_e2e / k_e2e * 1e6},
-        "gpu_launches": args.steps,
+        # per step: the fp16 copy of V, then the prefill kernel
+        "gpu_launches": 2 * args.steps,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": None,
-                     "kernel": "parallax_prefill_kernel", "peak_source": peak_src + " (burst)",
+                     "frac_of_sustained": achieved / sustained if sustained else None,
+                     "kernel": "parallax_prefill_kernel",
+                     "kernel_us_covers": "the fp16 copy of V and the prefill kernel",
+                     "peak_source": peak_src + " (burst)",
                      "kernel_us": kern_s * 1e6, "algorithmic_flops_per_launch": flops,
-                     "tensor_flops_issued_per_launch": flops // 8 * 12},
+                     "tensor_flops_issued_per_launch": flops},
         "cpu_baseline": cpu,
     }
     if dist.rank == 0:

@@ -282,17 +282,36 @@ int parallax_decode_block_sparse(const void* q, const void* r, const void* k_cac
  *  - D is 64 or 128; B and Hq at most 65535; scale positive and finite (the
  *    softmax temperature; PARALLAX_ERR_BAD_SHAPE otherwise).
  *  - The products Q K^T, R K^T, P V and (P o T) V run on the tcgen05 tensor
- *    cores (accumulators in tensor memory, P read from tensor memory); the
- *    weights e and e*s enter the value products as exact bf16 hi + lo pairs
- *    of their values rounded to 17 significant bits.
+ *    cores (accumulators in tensor memory, P read from tensor memory). The
+ *    weights e and e*s enter the value products as follows:
+ *      fp32 output: three bf16 terms each, which sum to the fp32 values exactly;
+ *      bf16 output, workspace of parallax_prefill_workspace_bytes(B, L, Hkv, D)
+ *      bytes or more: one fp16 term each (11 significant bits), against an fp16
+ *      copy of V that a kernel launched first writes into the workspace, on every
+ *      64-key tile whose V values are all below 2^16 in magnitude (fp16 holds
+ *      them exactly down to 2^-17, within 2^-25 below); e*s carries a power-of-
+ *      two factor per row, from a bound on |r . k|, that keeps it in fp16's
+ *      range. Other tiles, and every tile with a smaller workspace, take
+ *      bf16 hi + lo pairs of the weights rounded to 17 significant bits.
  *  - workspace: at least 256 bytes, zeroed once; its first word is the device
- *    status word read by parallax_workspace_status.
+ *    status word read by parallax_workspace_status. The rest (fp16 copy of V,
+ *    per-block records) is rewritten by every call, so concurrent calls need
+ *    separate workspaces.
  * Errors as parallax_decode.
  */
 int parallax_prefill(const void* q, const void* r, const void* k, const void* v,
                      void* out, int B, int Hq, int Hkv, int L, int D, float scale,
                      int causal, void* stream, int out_dtype, void* workspace,
                      size_t workspace_bytes);
+
+/*
+ * Workspace bytes with which a bf16-output parallax_prefill (dense: B batch
+ * rows of L keys) or parallax_varlen_prefill (B = 1, L = total_tokens) takes
+ * the fp16 value products: the 256-byte header, an fp16 copy of V
+ * (B * L * Hkv * D * 2 bytes from byte 1024) and 4 bytes per kv item and
+ * 64-key block. Returns 0 for B, L or Hkv below 1 or D other than 64 or 128.
+ */
+size_t parallax_prefill_workspace_bytes(int B, int L, int Hkv, int D);
 
 /*
  * The packed variable-length forward: parallax-kernel 0.1.0 README, "Helion
@@ -313,7 +332,8 @@ int parallax_prefill(const void* q, const void* r, const void* k, const void* v,
  *    written). 1 <= max_seqlen <= total_tokens.
  *  - Rows of a neighbouring sequence may be read into a tile and masked out
  *    (weight 0), so inputs must be finite.
- *  - workspace and errors as parallax_prefill.
+ *  - workspace and errors as parallax_prefill (the fp16 value products with
+ *    parallax_prefill_workspace_bytes(1, total_tokens, Hkv, D) bytes or more).
  */
 int parallax_varlen_prefill(const void* q, const void* r, const void* k, const void* v,
                             const int32_t* cu_seqlens, void* out, int B, int total_tokens,

@@ -97,7 +97,7 @@ def parallax_varlen_prefill(q, r, k, v, cu_seqlens, max_seqlen: Optional[int] = 
     if out is None:
         out = torch.empty_like(q, dtype=out_dtype if out_dtype is not None else q.dtype)
     if workspace is None:
-        workspace = torch.zeros(256, dtype=torch.uint8, device=q.device)
+        workspace = prefill_workspace(1, total, k.shape[1], D, q.device)
     buf = workspace.buffer if isinstance(workspace, Workspace) else workspace
     scale = D ** -0.5 if scale is None else scale
     rc = fn(q.data_ptr(), r.data_ptr(), k.data_ptr(), v.data_ptr(), cu_seqlens.data_ptr(),
@@ -445,6 +445,25 @@ def parallax_decode_noalloc(q, r, k_cache, v_cache, cache_seqlens, scale: Option
     return out
 
 
+def parallax_prefill_workspace_bytes(B: int, L: int, Hkv: int, D: int) -> int:
+    """Workspace bytes for the fp16 value products of a bf16-output prefill
+    (dense: B rows of L keys; packed: B = 1, L = total tokens)."""
+    lib = load_library()
+    fn = lib.parallax_prefill_workspace_bytes
+    fn.argtypes = [ctypes.c_int] * 4
+    fn.restype = ctypes.c_size_t
+    return int(fn(B, L, Hkv, D))
+
+
+def prefill_workspace(B: int, L: int, Hkv: int, D: int, device):
+    """A prefill workspace of parallax_prefill_workspace_bytes bytes with its
+    256-byte header (the status word) zeroed."""
+    ws = torch.empty(max(256, parallax_prefill_workspace_bytes(B, L, Hkv, D)), dtype=torch.uint8,
+                     device=device)
+    ws[:256].zero_()
+    return ws
+
+
 def parallax_prefill(q, r, k, v, scale: Optional[float] = None, causal: bool = True, out=None,
                      out_dtype=None, workspace=None, stream=None):
     """Training-shape forward (the README's parallax_func): q, r [B, Hq, L, D],
@@ -464,7 +483,7 @@ def parallax_prefill(q, r, k, v, scale: Optional[float] = None, causal: bool = T
     if out is None:
         out = torch.empty_like(q, dtype=out_dtype if out_dtype is not None else q.dtype)
     if workspace is None:
-        workspace = torch.zeros(256, dtype=torch.uint8, device=q.device)
+        workspace = prefill_workspace(B, L, Hkv, D, q.device)
     buf = workspace.buffer if isinstance(workspace, Workspace) else workspace
     scale = D ** -0.5 if scale is None else scale
     rc = fn(q.data_ptr(), r.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, Hq, Hkv,

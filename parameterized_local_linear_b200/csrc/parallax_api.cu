@@ -833,14 +833,14 @@ namespace {
 // items}: one box of `box_rows` rows x D dims lands as D/64 swizzled
 // [box_rows][128 bytes] blocks (the UMMA operand layout).
 int encode_rows_map(CUtensorMap* map, const void* base, int D, int L, long long items,
-                    int box_rows) {
+                    int box_rows, CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   auto enc = tensor_map_encoder();
   if (!enc) return PARALLAX_ERR_CUDA;
   cuuint64_t dims[4] = {64, (cuuint64_t)L, (cuuint64_t)(D / 64), (cuuint64_t)items};
   cuuint64_t strides[3] = {(cuuint64_t)D * 2, 128, (cuuint64_t)L * D * 2};
   cuuint32_t box[4] = {64, (cuuint32_t)box_rows, (cuuint32_t)(D / 64), 1};
   cuuint32_t elem[4] = {1, 1, 1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
+  CUresult r = enc(map, dtype, 4, const_cast<void*>(base), dims,
                    strides, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? PARALLAX_OK : PARALLAX_ERR_CUDA;
@@ -850,34 +850,87 @@ int encode_rows_map(CUtensorMap* map, const void* base, int D, int L, long long 
 // heads}: a box of `box_rows` consecutive rows of one head lands in the same
 // swizzled layout as encode_rows_map's.
 int encode_packed_map(CUtensorMap* map, const void* base, int D, int total, int H,
-                      int box_rows) {
+                      int box_rows, CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   auto enc = tensor_map_encoder();
   if (!enc) return PARALLAX_ERR_CUDA;
   cuuint64_t dims[4] = {64, (cuuint64_t)total, (cuuint64_t)(D / 64), (cuuint64_t)H};
   cuuint64_t strides[3] = {(cuuint64_t)H * D * 2, 128, (cuuint64_t)D * 2};
   cuuint32_t box[4] = {64, (cuuint32_t)box_rows, (cuuint32_t)(D / 64), 1};
   cuuint32_t elem[4] = {1, 1, 1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
+  CUresult r = enc(map, dtype, 4, const_cast<void*>(base), dims,
                    strides, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? PARALLAX_OK : PARALLAX_ERR_CUDA;
 }
 
+// Workspace of the bf16-output prefill: the 256-byte header, then (from byte
+// 1024) the fp16 copy of V, then one record per (kv item, 64-row block).
+// Dense: B batch rows of L keys, items = B * Hkv; packed: B = 1, L = total.
+struct PrefillWorkspace {
+  size_t v16_off, info_off, total;
+  int nblk;
+  long long items;
+};
+
+PrefillWorkspace prefill_workspace(int B, int L, int Hkv, int D) {
+  PrefillWorkspace w{};
+  w.nblk = (L + 63) / 64;
+  w.items = (long long)B * Hkv;
+  w.v16_off = 1024;
+  const size_t v16 = (size_t)B * (size_t)L * (size_t)Hkv * (size_t)D * 2;
+  w.info_off = w.v16_off + (v16 + 255) / 256 * 256;
+  w.total = w.info_off + (size_t)w.items * (size_t)w.nblk * 4;
+  return w;
+}
+
+// The fp16 copy of V and the per-block records, when the workspace holds
+// them (bf16 output only); then the prefill, chained with programmatic
+// dependent launch so that its set-up overlaps the end of the copy.
 template <int D, bool OUT_F32, bool VARLEN>
 int launch_prefill(const void* q, const void* r, const void* k, const void* v,
-                   const PrefillParams& prm, int grid_x, cudaStream_t stream) {
+                   PrefillParams prm, int grid_x, void* workspace, size_t workspace_bytes,
+                   cudaStream_t stream) {
   auto kernel = parallax_prefill_kernel<D, OUT_F32, VARLEN>;
   static std::atomic<int> done[256];
   int st = set_smem_once(kernel, PfGeom<D, OUT_F32>::kSmem, done);
   if (st != PARALLAX_OK) return st;
-  CUtensorMap tq, tr, tk, tv;
+  const int rows = VARLEN ? prm.total : prm.L;
+  const PrefillWorkspace w = prefill_workspace(VARLEN ? 1 : prm.B, rows, prm.Hkv, D);
+  const long long nprep = w.items * w.nblk;
+  const bool use16 = !OUT_F32 && workspace_bytes >= w.total && nprep <= 0x7fffffffLL;
+  char* const ws = static_cast<char*>(workspace);
+  CUtensorMap tq, tr, tk, tv, tv16;
   const void* src[4] = {q, r, k, v};
   CUtensorMap* maps[4] = {&tq, &tr, &tk, &tv};
   for (int i = 0; i < 4; ++i) {
-    const int H = i < 2 ? prm.Hq : prm.Hkv, rows = i < 2 ? kPfRows : kPfKeys;
-    st = VARLEN ? encode_packed_map(maps[i], src[i], D, prm.total, H, rows)
-                : encode_rows_map(maps[i], src[i], D, prm.L, (long long)prm.B * H, rows);
+    const int H = i < 2 ? prm.Hq : prm.Hkv, box = i < 2 ? kPfRows : kPfKeys;
+    st = VARLEN ? encode_packed_map(maps[i], src[i], D, prm.total, H, box)
+                : encode_rows_map(maps[i], src[i], D, prm.L, (long long)prm.B * H, box);
     if (st != PARALLAX_OK) return st;
+  }
+  tv16 = tv;
+  if (use16) {
+    st = VARLEN ? encode_packed_map(&tv16, ws + w.v16_off, D, prm.total, prm.Hkv, kPfKeys,
+                                    CU_TENSOR_MAP_DATA_TYPE_FLOAT16)
+                : encode_rows_map(&tv16, ws + w.v16_off, D, prm.L, (long long)prm.B * prm.Hkv,
+                                  kPfKeys, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+    if (st != PARALLAX_OK) return st;
+    prm.vinfo = reinterpret_cast<const uint32_t*>(ws + w.info_off);
+    prm.nblk = w.nblk;
+    dim3 grid((unsigned)w.nblk, 1, 1);
+    // one linear index would overflow gridDim.y's 65535 items: blocks in x, items in y and z
+    const long long items = w.items;
+    grid.y = (unsigned)std::min<long long>(items, 65535);
+    grid.z = (unsigned)((items + grid.y - 1) / grid.y);
+    if (grid.z > 65535) return PARALLAX_ERR_BAD_SHAPE;
+    parallax_prefill_prep_kernel<D, VARLEN><<<grid, 256, 0, stream>>>(
+        static_cast<const uint4*>(k), static_cast<const uint4*>(v),
+        reinterpret_cast<uint4*>(ws + w.v16_off), reinterpret_cast<uint32_t*>(ws + w.info_off),
+        rows, prm.Hkv, w.nblk, (int)grid.y, items);
+    if (cudaGetLastError() != cudaSuccess) return PARALLAX_ERR_CUDA;
+  } else {
+    prm.vinfo = nullptr;
+    prm.nblk = 0;
   }
   cudaLaunchConfig_t cfg = {};
   // one linear index over tile slots x Hq x B (slot slowest)
@@ -887,18 +940,27 @@ int launch_prefill(const void* q, const void* r, const void* k, const void* v,
   cfg.blockDim = dim3(kPfThreads);
   cfg.dynamicSmemBytes = PfGeom<D, OUT_F32>::kSmem;
   cfg.stream = stream;
-  return cudaLaunchKernelEx(&cfg, kernel, tq, tr, tk, tv, prm) == cudaSuccess ? PARALLAX_OK
-                                                                              : PARALLAX_ERR_CUDA;
+  cudaLaunchAttribute attr[1];
+  if (use16) {
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  return cudaLaunchKernelEx(&cfg, kernel, tq, tr, tk, tv, tv16, prm) == cudaSuccess
+             ? PARALLAX_OK
+             : PARALLAX_ERR_CUDA;
 }
 
 template <bool VARLEN>
 int dispatch_prefill(const void* q, const void* r, const void* k, const void* v,
-                     const PrefillParams& prm, int D, bool f32, int grid_x, cudaStream_t s) {
+                     const PrefillParams& prm, int D, bool f32, int grid_x, void* ws,
+                     size_t ws_bytes, cudaStream_t s) {
   if (D == 128)
-    return f32 ? launch_prefill<128, true, VARLEN>(q, r, k, v, prm, grid_x, s)
-               : launch_prefill<128, false, VARLEN>(q, r, k, v, prm, grid_x, s);
-  return f32 ? launch_prefill<64, true, VARLEN>(q, r, k, v, prm, grid_x, s)
-             : launch_prefill<64, false, VARLEN>(q, r, k, v, prm, grid_x, s);
+    return f32 ? launch_prefill<128, true, VARLEN>(q, r, k, v, prm, grid_x, ws, ws_bytes, s)
+               : launch_prefill<128, false, VARLEN>(q, r, k, v, prm, grid_x, ws, ws_bytes, s);
+  return f32 ? launch_prefill<64, true, VARLEN>(q, r, k, v, prm, grid_x, ws, ws_bytes, s)
+             : launch_prefill<64, false, VARLEN>(q, r, k, v, prm, grid_x, ws, ws_bytes, s);
 }
 
 // The checks both prefill layouts share.
@@ -944,7 +1006,8 @@ int run_prefill(const void* q, const void* r, const void* k, const void* v, void
   prm.timeout_ns = timeout_ns;
   prm.debug_skip_first_k = debug_skip_first_k;
   return dispatch_prefill<false>(q, r, k, v, prm, D, out_dtype == PARALLAX_DTYPE_F32,
-                                 prm.num_qt, static_cast<cudaStream_t>(stream));
+                                 prm.num_qt, workspace, workspace_bytes,
+                                 static_cast<cudaStream_t>(stream));
 }
 
 }  // namespace
@@ -955,6 +1018,11 @@ extern "C" int parallax_prefill(const void* q, const void* r, const void* k, con
                                 size_t workspace_bytes) {
   return run_prefill(q, r, k, v, out, B, Hq, Hkv, L, D, scale, causal, stream, out_dtype,
                      workspace, workspace_bytes, kDefaultTimeoutNs, 0);
+}
+
+extern "C" size_t parallax_prefill_workspace_bytes(int B, int L, int Hkv, int D) {
+  if (B < 1 || L < 1 || Hkv < 1 || (D != 64 && D != 128)) return 0;
+  return prefill_workspace(B, L, Hkv, D).total;
 }
 
 extern "C" int parallax_testing_prefill_stalled(const void* q, const void* r, const void* k,
@@ -993,7 +1061,7 @@ extern "C" int parallax_varlen_prefill(const void* q, const void* r, const void*
   prm.scale_log2 = (float)((double)scale * 1.4426950408889634);
   prm.timeout_ns = kDefaultTimeoutNs;
   return dispatch_prefill<true>(q, r, k, v, prm, D, out_dtype == PARALLAX_DTYPE_F32, prm.num_qt,
-                                static_cast<cudaStream_t>(stream));
+                                workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
 extern "C" int parallax_testing_decode_stalled(const void* q, const void* r, const void* k_cache,

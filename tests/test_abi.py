@@ -177,3 +177,16 @@ def test_split_env_override():
     assert run(base) == "148"
     assert run({**base, "PARALLAX_SPLITS": "37"}) == "37"
     assert run({**base, "PARALLAX_SPLITS": "junk"}) == "148"
+
+
+def test_prefill_workspace_bytes(lib):
+    """Header 256 B (padded to 1024), the fp16 copy of V, 4 bytes per (kv item,
+    64-key block); 0 for arguments outside the supported shapes."""
+    f = binding.parallax_prefill_workspace_bytes
+    B, L, Hkv, D = 4, 4096, 8, 128
+    v16 = B * L * Hkv * D * 2
+    assert f(B, L, Hkv, D) == 1024 + v16 + B * Hkv * (L // 64) * 4
+    # packed: one item per kv head over all tokens; a partial last block counts
+    assert f(1, 9991, 8, 64) == 1024 + (9991 * 8 * 64 * 2 + 255) // 256 * 256 + 8 * 157 * 4
+    for bad in ((0, 1, 1, 64), (1, 0, 1, 64), (1, 1, 0, 64), (1, 1, 1, 96)):
+        assert f(*bad) == 0

@@ -51,12 +51,14 @@ def test_bounded_wait_gives_up_and_context_survives():
     assert ws.status() == (0, 0)
 
 
-def test_prefill_bounded_wait_gives_up_and_context_survives():
+@pytest.mark.parametrize("ws_kind", ["header", "full"])
+def test_prefill_bounded_wait_gives_up_and_context_survives(ws_kind):
     """The tcgen05 prefill: the producer never loads a CTA's first K tile, so
     the UMMA issuer's wait runs out (50 ms); every CTA must record the timeout,
     drain its own copies, free its tensor memory and return, and a normal
     prefill on the same context (which allocates tensor memory again on every
-    SM) must then match the oracle."""
+    SM) must then match the oracle. 'full': with the workspace for the fp16
+    copy of V, so the stalled launch follows the copy kernel."""
     lib = binding.load_library()
     fn = lib.parallax_testing_prefill_stalled
     vp, i = ctypes.c_void_p, ctypes.c_int
@@ -68,7 +70,8 @@ def test_prefill_bounded_wait_gives_up_and_context_survives():
         torch.bfloat16)
     q, r, k, v = mk(Hq), mk(Hq, 0.5), mk(Hkv), mk(Hkv)
     out = torch.empty_like(q)
-    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    ws = (binding.prefill_workspace(B, L, Hkv, D, "cuda") if ws_kind == "full"
+          else torch.zeros(256, dtype=torch.uint8, device="cuda"))
     stream = torch.cuda.current_stream().cuda_stream
     t0 = time.perf_counter()
     rc = fn(q.data_ptr(), r.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, Hq, Hkv, L,
@@ -79,7 +82,7 @@ def test_prefill_bounded_wait_gives_up_and_context_survives():
     bits = int(ws[:4].view(torch.int32).item())
     assert bits & TIMEOUT_BIT, bits
     assert elapsed < 5.0, f"the stalled call took {elapsed:.2f} s"
-    ws.zero_()
+    ws[:256].zero_()
     got = binding.parallax_prefill(q, r, k, v, out_dtype=torch.float32, workspace=ws)
     want = oracle.parallax_prefill(q, r, k, v, D ** -0.5, True)
     gg = got.double().cpu().numpy()

@@ -32,21 +32,32 @@ def scaled_error(got, ref):
     return float(np.max(np.abs(g - ref) / np.maximum(1.0, np.abs(ref))))
 
 
+def workspace(kind, B, L, Hkv, D):
+    """'full': room for the fp16 copy of V (the fp16 value products with bf16
+    output); 'header': the 256-byte status header only (every tile takes the
+    bf16 hi + lo weights)."""
+    if kind == "full":
+        return binding.prefill_workspace(B, L, Hkv, D, "cuda")
+    return torch.zeros(256, dtype=torch.uint8, device="cuda")
+
+
+@pytest.mark.parametrize("ws_kind", ["full", "header"])
 @pytest.mark.parametrize("r_scale", [0.5, 1.0, 2.0])
 @pytest.mark.parametrize("L", [1, 64, 200, 384])
 @pytest.mark.parametrize("D", [64, 128])
 @pytest.mark.parametrize("Hq,Hkv", [(2, 2), (4, 2)])
-def test_prefill_matches_oracle(L, D, Hq, Hkv, r_scale):
+def test_prefill_matches_oracle(L, D, Hq, Hkv, r_scale, ws_kind):
     q, r, k, v = make(2, Hq, Hkv, L, D, seed=300 + L + D + Hq, r_scale=r_scale)
     scale = D ** -0.5
-    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    ws = workspace(ws_kind, 2, L, Hkv, D)
     for causal in (True, False):
         want = oracle.parallax_prefill(q, r, k, v, scale, causal)
         for out_dtype in (torch.bfloat16, torch.float32):
             got = binding.parallax_prefill(q, r, k, v, scale=scale, causal=causal,
                                            out_dtype=out_dtype, workspace=ws)
             err = scaled_error(got, want)
-            assert err <= TOL[out_dtype], (L, D, Hq, Hkv, r_scale, causal, out_dtype, err)
+            assert err <= TOL[out_dtype], (L, D, Hq, Hkv, r_scale, ws_kind, causal, out_dtype,
+                                           err)
     torch.cuda.synchronize()
     assert int(ws[:4].view(torch.int32).item()) == 0  # no device timeout
 
@@ -80,3 +91,42 @@ def test_prefill_full_size_sampled(r_scale):
         for dt, got in outs.items():
             err = scaled_error(got[b:b + 1, h:h + 1], want)
             assert err <= TOL[dt], (b, h, dt, r_scale, err)
+
+
+def row_scaled_error(got, ref):
+    """Error of each output over the largest |ref| of its row (at least 1).
+    With values of V in the hundreds of thousands the terms of
+    o = A/l + C/l - (b/l)(A/l) are ~1e6 and cancel: any fp32 evaluation is
+    off by units on the outputs of such a row that happen to be near zero,
+    so their error is measured against the row's magnitude."""
+    g = got.float().cpu().double().numpy()
+    assert np.all(np.isfinite(g)), "non-finite output"
+    scale = np.maximum(1.0, np.max(np.abs(ref), axis=-1, keepdims=True))
+    return float(np.max(np.abs(g - ref) / scale))
+
+
+@pytest.mark.parametrize("case", ["v_over_2e16", "v_near_f16_max", "probe_bound", "probe_huge",
+                                  "v_one_huge"])
+def test_prefill_tiles_outside_fp16_range(case):
+    """With bf16 output the value products take fp16 operands on tiles whose
+    V and probe-score bounds fit fp16, and the exact bf16 hi + lo weights on
+    the others; one sequence can mix both. Each case puts some tiles outside
+    the fp16 bounds (or right at their edge) and checks the result against
+    the oracle. A tile that took fp16 by mistake would turn V above 2^16
+    into inf; a row whose e*s were not scaled down would overflow fp16."""
+    B, Hq, Hkv, L, D = 1, 4, 2, 320, 128
+    q, r, k, v = make(B, Hq, Hkv, L, D, seed=340)
+    if case == "v_over_2e16":  # keys 64..127 of kv head 0 above fp16's range
+        v[:, 0, 64:128] = (v[:, 0, 64:128].float() * 3e5).to(torch.bfloat16)
+    elif case == "v_near_f16_max":  # in range, up to 65280 (exact in fp16)
+        v[:, 1, 128:192] = (v[:, 1, 128:192].float().clamp(-1, 1) * 65280).to(torch.bfloat16)
+    elif case == "probe_bound":  # |r|_1 max|k| above 2^14 for query heads 0 and 3: sigma > 0
+        r[:, 0] = (r[:, 0].float() * 400).to(torch.bfloat16)
+        r[:, 3] = (r[:, 3].float() * 400).to(torch.bfloat16)
+    elif case == "probe_huge":  # |s| itself beyond fp16's range, on some rows of head 1
+        r[:, 1, 100:140] = (r[:, 1, 100:140].float() * 2e4).to(torch.bfloat16)
+    else:  # one value of 1e6 in the middle of a tile, the rest of the row normal
+        v[:, 1, 200, 5] = 1e6
+    want = oracle.parallax_prefill(q, r, k, v, D ** -0.5, True)
+    got = binding.parallax_prefill(q, r, k, v, out_dtype=torch.bfloat16)
+    assert row_scaled_error(got, want) <= TOL[torch.bfloat16], case

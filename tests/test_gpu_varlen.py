@@ -38,21 +38,25 @@ def scaled_error(got, ref):
     return float(np.max(np.abs(g - ref) / np.maximum(1.0, np.abs(ref))))
 
 
+@pytest.mark.parametrize("ws_kind", ["full", "header"])
 @pytest.mark.parametrize("r_scale", [0.5, 1.0, 2.0])
 @pytest.mark.parametrize("D", [64, 128])
 @pytest.mark.parametrize("Hq,Hkv", [(2, 2), (4, 2)])
-def test_varlen_matches_oracle(D, Hq, Hkv, r_scale):
+def test_varlen_matches_oracle(D, Hq, Hkv, r_scale, ws_kind):
+    """'full': a workspace with room for the fp16 copy of V (fp16 value
+    products on in-range tiles, bf16 output); 'header': the status header only."""
     lens = [1, 130, 64, 0, 257, 5, 128]
     q, r, k, v, cu = make(lens, Hq, Hkv, D, seed=400 + D + Hq, r_scale=r_scale)
     scale = D ** -0.5
-    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    ws = (binding.prefill_workspace(1, sum(lens), Hkv, D, "cuda") if ws_kind == "full"
+          else torch.zeros(256, dtype=torch.uint8, device="cuda"))
     for causal in (True, False):
         want = oracle.parallax_varlen_prefill(q, r, k, v, cu, scale, causal)
         for out_dtype in (torch.bfloat16, torch.float32):
             got = binding.parallax_varlen_prefill(q, r, k, v, cu, max(lens), scale=scale,
                                                   causal=causal, out_dtype=out_dtype, workspace=ws)
             err = scaled_error(got, want)
-            assert err <= TOL[out_dtype], (D, Hq, Hkv, r_scale, causal, out_dtype, err)
+            assert err <= TOL[out_dtype], (D, Hq, Hkv, r_scale, ws_kind, causal, out_dtype, err)
     torch.cuda.synchronize()
     assert int(ws[:4].view(torch.int32).item()) == 0
 
