@@ -385,8 +385,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             umma_bf16(tmem + kPfColT, umma_smem_desc(sR + qo, 16, 1024),
                       umma_smem_desc(sKs + ko, 16, 1024), kIdescS, kk > 0);
           }
-          umma_commit(s_full);
-          umma_commit(k_empty + 8 * st);
+          umma_commit(s_full);  // also frees K_jj's stage: softmax warp 0 passes it on
         }
         if (jj >= 1) {  // O_A += P V, O_C += (P o T) V for tile j = jj - 1
           const int j = jj - 1, st = j % kSt;
@@ -436,8 +435,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                           true);
             }
           }
-          umma_commit(o_done);
-          umma_commit(v_empty + 8 * st);
+          umma_commit(o_done);  // also frees V_j's stage: softmax warp 0 passes it on
         }
       }
       if (!ok) {
@@ -510,6 +508,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(s_free);
+      // S_j, T_j complete: the score UMMAs have read K_j, so its stage can be
+      // refilled (an arrive here instead of a second commit by the issuer,
+      // each of which costs the tensor pipe ~50 ns)
+      if (warp == 0 && lane == 0) mbar_arrive(k_empty + 8 * (j % kSt));
       // causal mask (only tiles that reach past this tile's first row or the
       // end of the sequence need one) and the row max over all 64 keys
       const int k0 = j * kPfKeys, kown = k0 + 32 * half, kother = k0 + 32 * (half ^ 1);
@@ -552,6 +554,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                         mbar_wait_bounded(o_done, (j - 1) & 1, p.timeout_ns, abort_flag)))
           return false;
         tc_fence_after_sync();
+        // the value UMMAs of tile j - 1 have read V_{j-1}: its stage can be refilled
+        if (warp == 0 && lane == 0) mbar_arrive(v_empty + 8 * ((j - 1) % kSt));
         if (__any_sync(0xffffffffu, grow)) {  // warp-uniform: alpha is 1 on the other rows
           const uint32_t tO = tmem + lane_base + (half ? Geo::kColOC : Geo::kColOA);
 #pragma unroll 1
