@@ -105,17 +105,18 @@ def row_scaled_error(got, ref):
     return float(np.max(np.abs(g - ref) / scale))
 
 
+@pytest.mark.parametrize("D", [64, 128])
 @pytest.mark.parametrize("case", ["v_over_2e16", "v_near_f16_max", "probe_bound", "probe_huge",
                                   "v_one_huge"])
-def test_prefill_tiles_outside_fp16_range(case):
+def test_prefill_tiles_outside_fp16_range(case, D):
     """With bf16 output the value products take fp16 operands on tiles whose
     V and probe-score bounds fit fp16, and the exact bf16 hi + lo weights on
     the others; one sequence can mix both. Each case puts some tiles outside
     the fp16 bounds (or right at their edge) and checks the result against
     the oracle. A tile that took fp16 by mistake would turn V above 2^16
     into inf; a row whose e*s were not scaled down would overflow fp16."""
-    B, Hq, Hkv, L, D = 1, 4, 2, 320, 128
-    q, r, k, v = make(B, Hq, Hkv, L, D, seed=340)
+    B, Hq, Hkv, L = 1, 4, 2, 320
+    q, r, k, v = make(B, Hq, Hkv, L, D, seed=340 + D)
     if case == "v_over_2e16":  # keys 64..127 of kv head 0 above fp16's range
         v[:, 0, 64:128] = (v[:, 0, 64:128].float() * 3e5).to(torch.bfloat16)
     elif case == "v_near_f16_max":  # in range, up to 65280 (exact in fp16)
@@ -129,4 +130,4 @@ def test_prefill_tiles_outside_fp16_range(case):
         v[:, 1, 200, 5] = 1e6
     want = oracle.parallax_prefill(q, r, k, v, D ** -0.5, True)
     got = binding.parallax_prefill(q, r, k, v, out_dtype=torch.bfloat16)
-    assert row_scaled_error(got, want) <= TOL[torch.bfloat16], case
+    assert row_scaled_error(got, want) <= TOL[torch.bfloat16], (case, D)

@@ -115,3 +115,30 @@ def test_varlen_full_size_sampled():
                                                   np.array([0, e - a]), 128 ** -0.5)
             err = scaled_error(got[a:e, h:h + 1], want)
             assert err <= TOL[torch.float32], (s, h, err)
+
+
+def row_scaled_error(got, ref):
+    """Error over the largest |ref| of the row (at least 1): with values of V
+    in the hundreds of thousands, any fp32 evaluation of o is off by units on
+    outputs that happen to be near zero."""
+    g = got.float().cpu().double().numpy()
+    assert np.all(np.isfinite(g)), "non-finite output"
+    return float(np.max(np.abs(g - ref) / np.maximum(1.0, np.max(np.abs(ref), -1, keepdims=True))))
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_varlen_neighbour_rows_outside_fp16_range(D):
+    """A tile's K/V box can reach into the next sequence's rows, which are
+    masked (weight 0) but still multiplied. Here the second sequence's first
+    rows hold V above fp16's range: the first sequence's last tile, whose box
+    covers them, must not take the fp16 copy (inf times 0 would be NaN), and
+    the second sequence itself runs its first tile on the bf16 weights."""
+    lens = [100, 90, 200]
+    q, r, k, v, cu = make(lens, 4, 2, D, seed=460)
+    v[100:110] = (v[100:110].float() * 3e5).to(torch.bfloat16)  # rows 0..9 of sequence 1
+    want = oracle.parallax_varlen_prefill(q, r, k, v, cu, D ** -0.5, True)
+    ws = binding.prefill_workspace(1, sum(lens), 2, D, "cuda")
+    got = binding.parallax_varlen_prefill(q, r, k, v, cu, max(lens), workspace=ws)
+    assert row_scaled_error(got, want) <= TOL[torch.bfloat16]
+    torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32).item()) == 0
