@@ -134,3 +134,20 @@ def test_prefill_tiles_outside_fp16_range(case, D):
     want = oracle.parallax_prefill(q, r, k, v, D ** -0.5, True)
     got = binding.parallax_prefill(q, r, k, v, out_dtype=torch.bfloat16)
     assert row_scaled_error(got, want) <= TOL[torch.bfloat16], (case, D)
+
+
+def test_prefill_workspace_one_byte_short_takes_the_exact_weights():
+    """A workspace one byte smaller than parallax_prefill_workspace_bytes holds
+    no fp16 copy of V: every tile takes the bf16 hi + lo weights, and the call
+    matches the oracle within the fp32-accurate weights' error (well inside the
+    bf16 output's bound), as does the full workspace."""
+    B, Hq, Hkv, L, D = 1, 4, 2, 200, 128
+    q, r, k, v = make(B, Hq, Hkv, L, D, seed=350)
+    want = oracle.parallax_prefill(q, r, k, v, D ** -0.5, True)
+    n = binding.parallax_prefill_workspace_bytes(B, L, Hkv, D)
+    for size in (n - 1, n):
+        ws = torch.zeros(size, dtype=torch.uint8, device="cuda")
+        got = binding.parallax_prefill(q, r, k, v, out_dtype=torch.bfloat16, workspace=ws)
+        assert scaled_error(got, want) <= TOL[torch.bfloat16], size
+        torch.cuda.synchronize()
+        assert int(ws[:4].view(torch.int32).item()) == 0
