@@ -151,3 +151,68 @@ def test_prefill_workspace_one_byte_short_takes_the_exact_weights():
         assert scaled_error(got, want) <= TOL[torch.bfloat16], size
         torch.cuda.synchronize()
         assert int(ws[:4].view(torch.int32).item()) == 0
+
+
+def _expected_records(k, v, items_rows):
+    """Per (kv item, 64-row block): bits 0-15 the largest |k| as bf16 bits,
+    bit 16 set when every |v| is below 2^16 (a bf16 magnitude below 0x4780).
+    `items_rows` gives each item's rows as [rows, D] views."""
+    out = []
+    for kk, vv in items_rows(k, v):
+        kb = kk.contiguous().view(torch.int16).to(torch.int32) & 0x7FFF
+        vb = vv.contiguous().view(torch.int16).to(torch.int32) & 0x7FFF
+        rows = kb.shape[0]
+        for b0 in range(0, rows, 64):
+            km = int(kb[b0:b0 + 64].max())
+            ok = int(vb[b0:b0 + 64].max()) < 0x4780
+            out.append(km | (0x10000 if ok else 0))
+    return out
+
+
+@pytest.mark.parametrize("layout", ["dense", "packed"])
+@pytest.mark.parametrize("D", [64, 128])
+def test_prefill_prep_copy_and_records_are_exact(layout, D):
+    """The kernel launched before a bf16-output prefill writes, from byte 1024
+    of the workspace, V converted to fp16 (round to nearest even, inf at and
+    above 65520: the conversion torch performs) and, 256-byte aligned after
+    it, one 32-bit record per (kv item, 64-row block). Both are checked bit
+    for bit, on a V with one block out of fp16's range."""
+    Hq, Hkv = 4, 2
+    if layout == "dense":
+        B, L = 2, 200
+        q, r, k, v = make(B, Hq, Hkv, L, D, seed=360 + D)
+        v[1, 0, 70, 3] = 7e4  # item 2 (b = 1, g = 0), block 1
+        rows, items = L, B * Hkv
+        binding.parallax_prefill(q, r, k, v, out_dtype=torch.bfloat16,
+                                 workspace=(ws := binding.prefill_workspace(B, L, Hkv, D, "cuda")))
+        per_item = lambda kk, vv: [(kk[b, g], vv[b, g]) for b in range(B) for g in range(Hkv)]
+        v_elems = v.numel()
+    else:
+        lens = [130, 7, 200]
+        q, r, k, v, cu = _packed(lens, Hq, Hkv, D, seed=370 + D)
+        v[135, 1, 2] = -7e4  # head 1, packed row 135: block 2
+        rows, items = sum(lens), Hkv
+        ws = binding.prefill_workspace(1, rows, Hkv, D, "cuda")
+        binding.parallax_varlen_prefill(q, r, k, v, cu, max(lens), out_dtype=torch.bfloat16,
+                                        workspace=ws)
+        per_item = lambda kk, vv: [(kk[:, g], vv[:, g]) for g in range(Hkv)]
+        v_elems = v.numel()
+    torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32).item()) == 0
+    copy = ws[1024:1024 + 2 * v_elems].view(torch.float16).view(v.shape)
+    want = v.float().to(torch.float16)
+    assert torch.equal(copy.view(torch.int16), want.view(torch.int16))
+    info_off = 1024 + (2 * v_elems + 255) // 256 * 256
+    nblk = (rows + 63) // 64
+    rec = ws[info_off:info_off + 4 * items * nblk].view(torch.int32).cpu().tolist()
+    assert rec == _expected_records(k.cpu(), v.cpu(), per_item)
+    assert sum(1 for x in rec if not x & 0x10000) == 1  # the one out-of-range block
+
+
+def _packed(lens, Hq, Hkv, D, seed):
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    total = int(sum(lens))
+    rnd = lambda H: torch.randn(total, H, D, device="cuda", generator=g).to(torch.bfloat16)
+    q, r, k, v = rnd(Hq), rnd(Hq), rnd(Hkv), rnd(Hkv)
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32, device="cuda")
+    return q, r, k, v, cu
