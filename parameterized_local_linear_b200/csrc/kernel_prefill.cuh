@@ -484,10 +484,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           }
         }
         const float bound = rl1 * __uint_as_float(km << 16);
+        // 2^-sigma and 2^sigma stay normal floats for sigma <= 126, which covers
+        // every finite bound (below 2^128); an infinite bound (its product
+        // overflowed) takes 126, which brings any finite |s| below 4
         int sigma = 0;
         if (!(bound < 16384.f))  // also inf and NaN
-          sigma = bound < 3.0e38f ? (int)((__float_as_uint(bound) >> 23) & 0xffu) - 127 - 13 : 100;
-        sigma = min(max(sigma, 0), 100);
+          sigma = bound < 3.0e38f ? (int)((__float_as_uint(bound) >> 23) & 0xffu) - 127 - 13 : 126;
+        sigma = min(max(sigma, 0), 126);
         pt_scale = __int_as_float((127 - sigma) << 23);
         pt_unscale = __int_as_float((127 + sigma) << 23);
       }

@@ -12,7 +12,7 @@ parallax_prefill_workspace_bytes), checked over many shapes without a GPU:
 - the blocks a CTA scans for its bound on |k| cover every row of every box it
   loads;
 - sigma: the smallest power of two with |r|_1 max|k| 2^-sigma below 2^14
-  (clamped to 100 for inf and NaN), so that e*s 2^-sigma, with e <= 1, stays
+  (126 for inf and NaN; 2^-126 is still a normal float), so that e*s 2^-sigma, with e <= 1, stays
   far below fp16's largest value 65504.
 """
 import math
@@ -90,21 +90,22 @@ def sigma_of(bound):
             e = int((b.view(np.uint32) >> 23) & 0xFF) - 127
             sigma = e - 13
         else:
-            sigma = 100
+            sigma = 126
     else:
         sigma = 0
-    return min(max(sigma, 0), 100)
+    return min(max(sigma, 0), 126)
 
 
 def test_sigma_keeps_the_scaled_bound_below_2_14():
     rnd = random.Random(9)
-    values = [0.0, 1.0, 16383.0, 16384.0, 16385.0, 32767.0, 32768.0, 1e6, 3.3e38, float("inf"),
-              float("nan")] + [10 ** rnd.uniform(-3, 37) for _ in range(2000)]
+    values = [0.0, 1.0, 16383.0, 16384.0, 16385.0, 32767.0, 32768.0, 1e6, 2.15e35, 2.9e38, 3.3e38,
+              float("inf"), float("nan")] + [10 ** rnd.uniform(-3, 38.4) for _ in range(4000)]
     for bound in values:
         sigma = sigma_of(bound)
-        assert 0 <= sigma <= 100
+        assert 0 <= sigma <= 126
         if math.isnan(bound) or math.isinf(bound) or bound >= 3.0e38:
-            assert sigma == 100
+            assert sigma == 126
+            assert 3.4028235e38 * 2.0 ** -sigma < 4  # any finite |s|
             continue
         scaled = bound * 2.0 ** -sigma
         assert scaled < 16384.0, (bound, sigma)
