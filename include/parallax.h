@@ -226,13 +226,16 @@ int parallax_decode_plan(int B, int Hq, int Hkv, int D, int Lmax, int in_dtype, 
  *  - k_pages, v_pages [num_pages][page_size][Hkv][D] (a pool of pages), bf16
  *    or fp32 (in_dtype, which q and r share);
  *    block_table [B][max_pages_per_seq] int32: key i of sequence b is slot
- *    i % page_size of page block_table[b][i / page_size]. Only the entries a
- *    sequence's length reaches are read.
+ *    i % page_size of page block_table[b][i / page_size]. Entries past a
+ *    sequence's length may be read (the cluster schedule fetches a row's
+ *    first tiles before its length is known) but attend nothing, whatever
+ *    they hold.
  *  - page_size a multiple of 64 (every 64-key tile lies in one page);
  *    max_pages_per_seq * page_size plays the role of Lmax (cache_seqlens are
  *    clamped to it; NULL lengths mean that many keys).
- *  - A page id outside [0, num_pages) is not read: its keys are left out and
- *    PARALLAX_DEVICE_STATUS_SEQLEN_CLAMPED is set.
+ *  - A page id outside [0, num_pages) is not read: its keys are left out and,
+ *    for an entry the length reaches, PARALLAX_DEVICE_STATUS_SEQLEN_CLAMPED
+ *    is set.
  *  - probe != 0: the Parallax output (r required); probe == 0: R = 0 softmax.
  *  - bf16 or fp32 inputs (in_dtype); any query-head group. bf16 pools with
  *    up to 4 query heads per kv head with the probe (8 without) run on the

@@ -144,12 +144,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   pdl_wait_primary();
 
   // tile j of this CTA is the item's tile rank + S j; on a contiguous row
-  // without a window the first ones that fit in the ring and lie inside the
-  // cache are issued before the length is known
+  // without a window, and on a paged row, the first ones that fit in the ring
+  // and lie inside the row's capacity are issued before the length is known
+  // (a paged tile's page id and attended prefix come with it from tile_source;
+  // one past the length attends nothing)
   const KeySpace ks = key_space(p);
   const bool contiguous = p.kv_mode == kKvContiguous;
   const int cache_tiles = (p.Lmax + kTileKeys - 1) / kTileKeys;
-  const int nspec = (contiguous && p.window == 0 && rank < cache_tiles)
+  const bool speculate = (contiguous && p.window == 0) || p.kv_mode == kKvPaged;
+  const int nspec = (speculate && rank < cache_tiles)
                         ? min(kStages, (cache_tiles - rank + S - 1) / S)
                         : 0;
   const bool skip0 = p.debug_skip_first_tile != 0;  // testing hook: stage 0 never filled

@@ -230,7 +230,9 @@ __device__ __forceinline__ void tile_source(const Params& p, int b, int k0, int*
     *key = ok ? k0 % p.page_size : 0;
     *item = ok ? page : 0;
     *nv = ok ? max(0, min(kRangeAlign, n - k0)) : 0;
-    if (!ok) atomicOr(p.status, 2u /* PARALLAX_DEVICE_STATUS_SEQLEN_CLAMPED */);
+    // an entry past the length (read when the cluster kernel fetches a row's
+    // first tiles before its length) attends nothing and is not an error
+    if (!ok && k0 < n) atomicOr(p.status, 2u /* PARALLAX_DEVICE_STATUS_SEQLEN_CLAMPED */);
   } else {  // block-sparse: the listed block of the cache row
     const int blk = __ldg(p.table + (size_t)b * p.table_stride + k0 / kRangeAlign);
     const bool ok = blk >= 0 && (long long)blk * kRangeAlign < p.Lmax;

@@ -101,6 +101,34 @@ def test_paged_without_lengths_and_bad_page():
     assert scaled_error(got[0], want[0]) <= 1e-4  # the other sequence is untouched
 
 
+@pytest.mark.parametrize("page_size", [64, 256])
+def test_paged_entries_past_the_length_are_ignored(page_size):
+    """The cluster schedule (few items, num_splits = 0) fetches a row's first
+    tiles before its length is known, so it reads table entries past the
+    length. Whatever they hold (ids outside the pool here, or -1), those keys
+    attend nothing and no status bit is set; an out-of-range id the length
+    reaches still sets it."""
+    max_pages = 2048 // page_size
+    lens = [1, 300, 2048]
+    q, r, kp, vp, table, n = paged_case(540 + page_size, 3, 16, 8, 128, page_size, max_pages,
+                                        lens)
+    for b, nb in enumerate(lens):
+        used = (nb + page_size - 1) // page_size
+        table[b, used:] = -1 if b % 2 else kp.shape[0] + 1000
+    want = oracle.parallax_decode_paged(q, r, kp, vp, table, n, 128 ** -0.5)
+    assert binding.parallax_decode_plan(3, 16, 8, 128, max_pages * page_size)["cluster_ctas"] > 0
+    ws = binding.Workspace(3, 16, 8, 128, max_pages * page_size)
+    for out_dtype in (torch.bfloat16, torch.float32):
+        got = binding.parallax_decode_paged(q, r, kp, vp, table, n, out_dtype=out_dtype,
+                                            workspace=ws)
+        assert scaled_error(got, want) <= TOL[out_dtype], out_dtype
+        assert status_bits(ws) == 0
+    bad = table.clone()
+    bad[1, 0] = kp.shape[0] + 3  # the length reaches this one
+    binding.parallax_decode_paged(q, r, kp, vp, bad, n, workspace=ws)
+    assert status_bits(ws) & 2
+
+
 def sparse_case(seed, B, Hq, Hkv, D, Lmax, lens, layout, dtype=torch.bfloat16):
     g = torch.Generator(device="cuda").manual_seed(seed)
     q = torch.randn(B, Hq, D, device="cuda", generator=g).to(dtype)
