@@ -129,3 +129,26 @@ def test_reduction_lanes_stay_in_whole_warps():
                     first = base + (lane // W) * W
                     assert divmod(first, W)[0] == j and first // 32 == idx // 32
                     assert src < W
+
+
+@pytest.mark.parametrize("page_size", [64, 128, 256, 1024])
+def test_paged_speculative_tiles_stay_in_the_table_row(page_size):
+    """Paged rows fetch their first tiles before the length is known: tile j of
+    CTA `rank` is row position (rank + S j) * 64, and its page id is entry
+    position / page_size of the row's table. With Lmax = max_pages *
+    page_size, every speculative tile reads an entry inside the row (never
+    the next row's), and a tile at or past the length attends nothing."""
+    for D in (64, 128):
+        stages = STAGES[D]
+        for S, max_pages, n in itertools.product(range(2, 17), (1, 2, 3, 16, 64),
+                                                 (0, 1, 64, 200, 4096)):
+            Lmax = max_pages * page_size
+            n = min(n, Lmax)
+            cache_tiles = (Lmax + TILE - 1) // TILE
+            for rank in range(S):
+                nspec = min(stages, (cache_tiles - rank + S - 1) // S) if rank < cache_tiles else 0
+                for j in range(nspec):
+                    k0 = (rank + S * j) * TILE
+                    assert 0 <= k0 // page_size < max_pages
+                    attended = max(0, min(TILE, n - k0))
+                    assert (attended == 0) == (k0 >= n)
